@@ -1,0 +1,428 @@
+#!/usr/bin/env python3
+"""Benchmark of the SAS gated block-sparse attention hot path on B200.
+
+One step is one pass of the training hot path over the Qwen3-4B-shaped
+workload: batch 1, 32 query / 8 KV heads, d 128, 32768 tokens, block 64,
+Top-K 32. It runs Top-K selection + LSE(s), the gated forward, and the
+backward with dq/dk/dv and the score gradient ds. The headline value is
+selected-token TFLOP/s for fwd+bwd. The FLOP rule, per query head and query
+block, is fwd = 4·d·64·(64·n_t + 32) and bwd = 2.5·fwd, where n_t = min(K, t)
+and the causal current block counts as half.
+
+The same JSON line also reports the single-token decode workload (16
+sequences with 32768-token caches, Top-K 16 plus the current block, split-K +
+merge) as tokens/s and gathered-KV GB/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 the script runs under torch.distributed.run, one rank per GPU.
+Every rank processes its own replica of the workload (independent sequences,
+no collective on the data path). value = total FLOPs of all ranks ÷ the
+slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated block-sparse attn TFLOP/s fwd+bwd and decode tok/s; % of roofline"
+TRAIN = "qwen3_4b_train_32k"
+DECODE = "decode_b16_32k"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# work counts
+# ---------------------------------------------------------------------------
+def fwd_flops(n_q_heads, head_dim, n_blocks, top_k, batch=1, block=64, t_list=None):
+    ts = range(n_blocks) if t_list is None else t_list
+    per_head = sum(4.0 * head_dim * block * (block * min(top_k, t) + block / 2) for t in ts)
+    return per_head * n_q_heads * batch
+
+
+def decode_kv_bytes(w, cache_len):
+    n_blocks = 0
+    for L in cache_len:
+        c = (int(L) - 1) // w.block
+        n_blocks += min(w.top_k, c) * w.block + (int(L) - c * w.block)
+    return n_blocks * w.n_kv_heads * w.head_dim * 2 * 2  # K and V, bf16
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return dict(bf16=m["bf16_tflops"], bf16_sustained=m.get("bf16_tflops_sustained", m["bf16_tflops"]),
+                    hbm=m["hbm_gbs"], source="measured")
+    return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def traffic_record(kernel_key, src_files):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel_key)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for s in src_files:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    return rec["bytes_per_launch"] if rec.get("source_sha256") == h.hexdigest() else None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample
+# ---------------------------------------------------------------------------
+def oracle_baseline(w, budget_s=15.0):
+    """Times the oracle's fwd+bwd on one KV head over a growing set of query blocks."""
+    import oracle.sas_oracle as O
+    from synth import workloads as W
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    x = W.prefill_inputs(w, kv_heads=[0])
+    idx, _ = O.prefill_select(x["s"].astype(np.float64), w.top_k)
+    NB = w.n_blocks
+    order = list(range(NB - 1, -1, -max(1, NB // 64)))  # spread over the sequence, long rows first
+    done, t_used, flops = [], 0.0, 0.0
+    t0 = time.perf_counter()
+    for t in order:
+        a = time.perf_counter()
+        O.backward(x["q"], x["k"], x["v"], x["s"], idx, x["do"], t_list=[t])  # recomputes P and o itself
+        O.forward(x["q"], x["k"], x["v"], x["s"], idx, t_list=[t])
+        t_used += time.perf_counter() - a
+        done.append(t)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    flops = 3.5 * fwd_flops(w.group, w.head_dim, NB, w.top_k, t_list=done)
+    return {"value": flops / t_used / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"KV head 0 ({w.group} query heads), {len(done)} of {NB} query blocks spread over the "
+                      f"sequence, fwd+bwd in NumPy fp64; {t_used:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import learned_block_sparse_warp_b200 as sas
+    from synth import workloads as W
+    from synth.device import decode_to_device, prefill_to_device
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.Stream(device=dev)
+    w = W.WORKLOADS[TRAIN]
+    p = sas.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
+                   seq_len=w.seq_len, top_k=w.top_k, gate_mode=sas.SAS_GATE_LOG_SOFTMAX)
+    x = prefill_to_device(w, device=dev)
+    out = sas.empty_prefill_outputs(p, device=dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
+
+    def step(q, k, v, s, dO, o):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        sas.sas_topk_select(p, s, o["idx"], o["lse_s"], stream=stream)
+        ev[1].record(stream)
+        sas.sas_fwd(p, q, k, v, s, o["idx"], o["lse_s"], o["o"], o["lse_o"], stream=stream)
+        ev[2].record(stream)
+        sas.sas_bwd(p, q, k, v, o["o"], dO, s, o["idx"], o["lse_s"], o["lse_o"], o["dq"], o["dk"], o["dv"],
+                    o["ds"], o["ws"], stream=stream)
+        ev[3].record(stream)
+        return ev
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step(x["q"], x["k"], x["v"], x["s"], x["do"], out)
+    torch.cuda.synchronize()
+    if sas.sas_get_device_error(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    barrier()
+    torch.cuda.synchronize()
+    evs = []
+    with ClockSampler(local_rank) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for _ in range(args.steps):
+            evs.append(step(x["q"], x["k"], x["v"], x["s"], x["do"], out))
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    F = fwd_flops(w.n_q_heads, w.head_dim, w.n_blocks, w.top_k, batch=w.batch)
+    step_flops = 3.5 * F
+    ms_per_step = total_ms / args.steps
+    value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
+    pk = peaks()
+
+    # end to end through the public API: pinned host inputs in, every output back to pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        h_in = {k_: t.cpu().pin_memory() for k_, t in x.items()}
+        d_in = {k_: torch.empty_like(t) for k_, t in x.items()}
+        outs = ["o", "lse_o", "dq", "dk", "dv", "ds"]
+        h_out = {k_: torch.empty(out[k_].shape, dtype=out[k_].dtype, pin_memory=True) for k_ in outs}
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for k_ in d_in:
+                    d_in[k_].copy_(h_in[k_], non_blocking=True)
+                step(d_in["q"], d_in["k"], d_in["v"], d_in["s"], d_in["do"], out)
+                for k_ in outs:
+                    h_out[k_].copy_(out[k_], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, min(args.steps, 3))
+        barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b)) / n_e2e
+        e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e}
+        del h_in, d_in, h_out
+
+    # decode workload: split-K + merge, L2 flushed before every timed step
+    dec = None
+    if not args.no_decode:
+        del x
+        wd = W.WORKLOADS[DECODE]
+        pd = sas.Params(batch=wd.batch, n_q_heads=wd.n_q_heads, n_kv_heads=wd.n_kv_heads, head_dim=wd.head_dim,
+                        seq_len=wd.seq_len, top_k=wd.top_k, gate_mode=sas.SAS_GATE_NONE)
+        xd = decode_to_device(wd, device=dev)
+        n_split = wd.top_k + 1
+        od = sas.empty_decode_outputs(pd, n_split, device=dev)
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+        def dstep():
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
+            sas.sas_topk_select(pd, xd["s"], od["idx"], od["lse_s"], cache_len=xd["cache_len"], stream=stream)
+            ev[1].record(stream)
+            sas.sas_decode(pd, xd["q"], xd["k"], xd["v"], xd["cache_len"], xd["s"], od["idx"], od["lse_s"],
+                           n_split, od["o_part"], od["lse_part"], stream=stream)
+            ev[2].record(stream)
+            sas.sas_decode_combine(pd, n_split, od["o_part"], od["lse_part"], od["o"], od["lse_o"], stream=stream)
+            ev[3].record(stream)
+            return ev
+
+        n_dec = max(20, args.steps * 4)
+        dev_evs = []
+        with torch.cuda.stream(stream):
+            for _ in range(max(3, args.warmup)):
+                dstep()
+            for _ in range(n_dec):
+                flush.zero_()
+                dev_evs.append(dstep())
+        torch.cuda.synchronize()
+        step_ms = statistics.median(e[0].elapsed_time(e[3]) for e in dev_evs)
+        split_ms = statistics.median(e[1].elapsed_time(e[2]) for e in dev_evs)
+        sel_d_ms = statistics.median(e[0].elapsed_time(e[1]) for e in dev_evs)
+        comb_ms = statistics.median(e[2].elapsed_time(e[3]) for e in dev_evs)
+        step_ms = max_over_ranks(step_ms)
+        kv = decode_kv_bytes(wd, xd["cache_len"].cpu().numpy())
+        gbs = kv / (split_ms * 1e-3) / 1e9
+        dec = {"workload": DECODE, "tok_per_s": world * wd.batch / (step_ms * 1e-3), "ms_per_step": step_ms,
+               "select_ms": sel_d_ms, "split_ms": split_ms, "combine_ms": comb_ms, "n_split": n_split,
+               "gate": "none (inference form)", "l2": "flushed (512 MB write) before every step",
+               "roofline": {"bound": "hbm", "kernel": "decode_split_kernel (sas_decode)", "achieved": gbs,
+                            "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
+                            "algorithmic_bytes": kv,
+                            "traffic": traffic_record("decode_split", ["learned_block_sparse_warp_b200/csrc/decode.cu"])},
+               "gpu_launches_per_step": 3}
+        if sas.sas_get_device_error(stream) != 0:
+            raise RuntimeError("device error during decode")
+
+    bwd_flops = 2.5 * F
+    achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": TRAIN, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                   "head_dim": w.head_dim, "seq_len": w.seq_len, "block": w.block, "top_k": w.top_k,
+                   "gate": "log_softmax (training form)", "flops_per_step": step_flops,
+                   "parallelism": f"dp{world} (independent replicas)",
+                   "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > 126 MB L2 (no flush)"},
+        "breakdown_ms": {"select": sel_ms, "fwd": fwd_ms, "bwd": bwd_ms},
+        "fwd_tflops": F / (fwd_ms * 1e-3) / 1e12,
+        "bwd_tflops": achieved,
+        "roofline": {"bound": "tensor", "kernel": "sas_bwd call (bwd_main_kernel + prep/reverse-index/epilogue)",
+                     "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_sustained"], "peak_source": pk["source"] + " sustained bf16",
+                     "traffic": traffic_record("bwd_main", ["learned_block_sparse_warp_b200/csrc/bwd_mma.cu"])},
+        "e2e": e2e,
+        "gpu_launches": args.steps * 9,
+        "clocks": clk.summary(),
+    }
+    if dec is not None:
+        line["decode"] = dec
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline(w, budget_s=args.cpu_budget)
+    if dist is not None:
+        dist.destroy_process_group()
+    return line
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from synth import workloads as W
+    w = W.WORKLOADS[TRAIN]
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_baseline(w, budget_s=budget)
+    vals = []
+    cb = None
+    for _ in range(args.steps):
+        cb = oracle_baseline(w, budget_s=budget)
+        vals.append(cb["value"])
+    value = statistics.mean(vals)
+    F = fwd_flops(w.n_q_heads, w.head_dim, w.n_blocks, w.top_k)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 3.5 * F / (value * 1e12) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": TRAIN, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                       "head_dim": w.head_dim, "seq_len": w.seq_len, "block": w.block, "top_k": w.top_k,
+                       "gate": "log_softmax (training form)"},
+            "cpu_baseline": dict(cb, value=value),
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["sas", "reference"], default="sas")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus:
+        world = args.gpus if "WORLD_SIZE" not in os.environ else world
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_gpu(args, rank, world, local_rank)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,226 @@
+/*
+ * sas.h — C ABI of the SAS gated block-sparse attention library for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The method: the context is cut into blocks of b = 64 tokens. A selector
+ * gives one score s_m per history block. Every query block keeps its own
+ * block B0, causally masked and with gate 1. It also keeps the Top-K history
+ * blocks by s. For training, the softmax-normalised gate goes inside the
+ * attention softmax as log g_m = s_m − LSE(s):
+ *
+ *     o = softmax(q K_Sᵀ·scale + log g_S) V_S,   S = B0 ∪ ⋃_{m∈I} B_m.
+ *
+ * Sources:
+ *  - SAS explainer (ta-paperlens, "論文解説: SAS — 疎注意の「どのブロックを
+ *    読むか」を言語モデル損失で端から端まで学習する"). §前提 covers blocks,
+ *    Top-K and the union S. §仕組み covers the gate, Eq. (9) and the ungated
+ *    inference form (Algorithm 2).
+ *  - SAS summary (onedev.kr, "SAS는 언어모델 손실로 문맥 순위를 직접 학습하는
+ *    사후 어텐션 희소화다."). §어떻게 동작하나 gives o_SAS. §무엇과 다른가
+ *    gives g = softmax(s), log g_m = s_m − LSE(s), the gate gradient
+ *    dg_m = Σ_i (p̃_i/g_m) dOᵀ(v_i − o) and sparse-scope training.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    allocates no device memory. The only host pointers are `p`, the `bytes`
+ *    output of sas_bwd_workspace_size and the `code` output of
+ *    sas_get_device_error.
+ *  - Tensors are dense, row-major, in the stated layouts. The last dimension
+ *    is innermost. Every tensor pointer must be 16-byte aligned.
+ *  - bf16 tensors hold IEEE bfloat16 bit patterns (sas_bf16 = uint16_t).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL means the
+ *    legacy default stream). Arguments are checked on the host before any
+ *    launch. A bad argument returns an error status and launches nothing.
+ *    A launch failure returns SAS_ERR_CUDA. Device-side faults that the
+ *    kernels detect themselves are raised through sas_get_device_error, for
+ *    example an index outside the history or a bounded wait that expired.
+ *  - Calls keep no state between them and may be issued from several host
+ *    threads, on different streams.
+ *
+ * Shapes (sas_params): B = batch, Hq = n_q_heads, Hkv = n_kv_heads,
+ * G = Hq / Hkv (GQA group), d = head_dim, N = seq_len, b = block (64),
+ * NQB = NKB = N / b, K = top_k. Query block t covers tokens [b·t, b·t + b).
+ * Its history is blocks 0..t−1, and it selects n_t = min(K, t) of them.
+ */
+#ifndef SAS_H_
+#define SAS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAS_API __attribute__((visibility("default")))
+#else
+#define SAS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t sas_bf16;
+
+typedef enum {
+  SAS_OK = 0,
+  SAS_ERR_INVALID_ARG = 1, /* a pointer, size or layout rule is broken */
+  SAS_ERR_UNSUPPORTED = 2, /* valid, but no kernel for it (e.g. head_dim 96) */
+  SAS_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+  SAS_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  SAS_ERR_TIMEOUT = 5,     /* a device-side bounded wait expired */
+  SAS_ERR_DEVICE_INDEX = 6 /* a kernel met a block index outside the history */
+} sas_status;
+
+typedef enum {
+  /* Training form, Eq. (9): log g_m = s_m − LSE(s) is added to the logits of
+   * every token of selected history block m. The current block gets 0. */
+  SAS_GATE_LOG_SOFTMAX = 0,
+  /* Inference form (Algorithm 2): Top-K selection only, no gate term. */
+  SAS_GATE_NONE = 1
+} sas_gate_mode;
+
+typedef struct {
+  int batch;           /* B >= 1 */
+  int n_q_heads;       /* Hq >= 1, a multiple of n_kv_heads */
+  int n_kv_heads;      /* Hkv >= 1 */
+  int head_dim;        /* d: 64 or 128 */
+  int seq_len;         /* prefill: N; decode: KV-cache capacity Lmax; a multiple of block */
+  int block;           /* b: must be 64 */
+  int top_k;           /* K: 1..256 */
+  float softmax_scale; /* 0 selects 1/sqrt(d) */
+  int gate_mode;       /* sas_gate_mode */
+} sas_params;
+
+/* ---------------------------------------------------------------------------
+ * Selection and gate normaliser
+ * SAS explainer §前提: Top-K of the history scores. SAS summary §무엇과 다른가:
+ * LSE(s) is the normaliser of g = softmax(s).
+ * ------------------------------------------------------------------------- */
+
+/* Top-K history blocks of every query block, and optionally LSE(s).
+ *
+ * Prefill form (cache_len == NULL):
+ *   s       fp32  [B, Hkv, NQB, NKB]. Only entries m < t of row t are read.
+ *   idx     int32 [B, Hkv, NQB, K]. Output. The n_t = min(K, t) blocks with
+ *           the highest s[t, m] for m < t, ties to the lower m, written in
+ *           ascending m. Slots n_t..K−1 hold −1.
+ *   lse_s   fp32  [B, Hkv, NQB]. Output, may be NULL.
+ *           lse_s[t] = log Σ_{m<t} exp s[t, m], and −inf at t = 0.
+ * Decode form (cache_len != NULL):
+ *   cache_len int32 [B]. Tokens in each sequence's cache, the new token
+ *           included, 1 <= L <= seq_len. The current block is c = (L−1)/b.
+ *           History is blocks 0..c−1.
+ *   s       fp32  [B, Hkv, NKB]. Only m < c is read.
+ *   idx     int32 [B, Hkv, K]; lse_s fp32 [B, Hkv] (may be NULL).
+ * Scores must be finite. NaN ranks below every number. */
+SAS_API sas_status sas_topk_select(const sas_params* p, const float* s, const int32_t* cache_len, int32_t* idx,
+                           float* lse_s, void* stream);
+
+/* LSE(s) alone, with the same layouts and forms as sas_topk_select. */
+SAS_API sas_status sas_gate_lse(const sas_params* p, const float* s, const int32_t* cache_len, float* lse_s,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Forward, Eq. (9) (SAS explainer §仕組み; SAS summary §어떻게 동작하나)
+ * ------------------------------------------------------------------------- */
+
+/* o_i = Σ_{j∈S_t} softmax_j(z_ij) v_j with z_ij = scale·q_i·k_j + λ_j.
+ * λ_j = s[t, m(j)] − lse_s[t] for tokens of the selected history blocks
+ * (SAS_GATE_LOG_SOFTMAX) and 0 for the current block. In the current block,
+ * column j is visible to row i only when j <= i.
+ *   q      bf16 [B, Hq, N, d]
+ *   k, v   bf16 [B, Hkv, N, d]
+ *   s      fp32 [B, Hkv, NQB, NKB]. Read only under SAS_GATE_LOG_SOFTMAX.
+ *   idx    int32 [B, Hkv, NQB, K], as written by sas_topk_select.
+ *   lse_s  fp32 [B, Hkv, NQB]. Required under SAS_GATE_LOG_SOFTMAX,
+ *          ignored (may be NULL) under SAS_GATE_NONE.
+ *   o      bf16 [B, Hq, N, d]. Output.
+ *   lse_o  fp32 [B, Hq, N]. Output, may be NULL. Row log-sum-exp of z,
+ *          which the backward needs.
+ * An idx entry outside [0, t) is skipped and raises SAS_ERR_DEVICE_INDEX. */
+SAS_API sas_status sas_fwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, const sas_bf16* v, const float* s,
+                   const int32_t* idx, const float* lse_s, sas_bf16* o, float* lse_o, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Backward with the gate/score gradient (SAS summary §무엇과 다른가: the gate
+ * inside the softmax, chained through g = softmax(s); sparse scope)
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device workspace that sas_bwd needs for these params. */
+SAS_API sas_status sas_bwd_workspace_size(const sas_params* p, size_t* bytes);
+
+/* Gradients of ⟨dO, o⟩ with the selection idx held fixed.
+ *   Inputs: q, k, v, s, idx, lse_s as in sas_fwd. o and lse_o are the
+ *   forward's outputs. dO is bf16 [B, Hq, N, d].
+ *   dq     bf16 [B, Hq, N, d]. Output.
+ *   dk, dv bf16 [B, Hkv, N, d]. Output. Summed over the G query heads.
+ *   ds     fp32 [B, Hkv, NQB, NKB]. Output. With dl[t, m] the gradient for
+ *          log g_m summed over block m's tokens, the rows of query block t and
+ *          the G heads,
+ *            ds[t, m] = dl[t, m]·[m ∈ I_t] − softmax(s[t, 0:t])_m · Σ_{m'∈I_t} dl[t, m'].
+ *          Zero for m >= t, and zero everywhere under SAS_GATE_NONE. May be
+ *          NULL under SAS_GATE_NONE.
+ *   ws     device workspace of at least sas_bwd_workspace_size bytes,
+ *          256-byte aligned. Its contents on entry do not matter. The call
+ *          overwrites it.
+ * idx must be in the form sas_topk_select writes: ascending, −1 padded.
+ * Other index lists are memory-safe but their gradients are unspecified. */
+SAS_API sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, const sas_bf16* v,
+                   const sas_bf16* o, const sas_bf16* dO, const float* s, const int32_t* idx, const float* lse_s,
+                   const float* lse_o, sas_bf16* dq, sas_bf16* dk, sas_bf16* dv, float* ds, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Split-K single-token decode (SAS explainer §仕組み: at inference Top-K on s,
+ * then ordinary sparse attention; SAS summary §전제와 한계: decode is the
+ * sparsified stage)
+ * ------------------------------------------------------------------------- */
+
+/* One new query token per sequence, at position L−1 with L = cache_len[b].
+ * It attends to the current block c = (L−1)/b, whose tokens b·c..L−1 carry
+ * gate 1, and to the selected history blocks idx[b, h, 0..n−1], n = min(K, c).
+ * Under SAS_GATE_LOG_SOFTMAX those blocks get λ = s − lse_s. The ordered
+ * block list [c, idx...] is cut into n_split contiguous chunks of
+ * ceil((n+1)/n_split) blocks. Split j covers its chunk and writes that
+ * chunk's normalised output and log-sum-exp. An empty chunk gives o = 0 and
+ * lse = −inf.
+ *   q          bf16 [B, Hq, d]
+ *   kc, vc     bf16 [B, Hkv, Lmax, d]   (Lmax = seq_len)
+ *   cache_len  int32 [B], 1 <= L <= Lmax
+ *   s          fp32 [B, Hkv, NKB]. Read only under SAS_GATE_LOG_SOFTMAX.
+ *   idx        int32 [B, Hkv, K] from sas_topk_select (decode form)
+ *   lse_s      fp32 [B, Hkv]. Required under SAS_GATE_LOG_SOFTMAX.
+ *   n_split    1..K+1
+ *   o_part     fp32 [B, Hq, n_split, d]. Output.
+ *   lse_part   fp32 [B, Hq, n_split]. Output. */
+SAS_API sas_status sas_decode(const sas_params* p, const sas_bf16* q, const sas_bf16* kc, const sas_bf16* vc,
+                      const int32_t* cache_len, const float* s, const int32_t* idx, const float* lse_s, int n_split,
+                      float* o_part, float* lse_part, void* stream);
+
+/* Merge of the split partials:
+ *   LSE = log Σ_j exp lse_part[j],   o = Σ_j exp(lse_part[j] − LSE) · o_part[j].
+ *   o      bf16 [B, Hq, d]. Output.
+ *   lse_o  fp32 [B, Hq]. Output, may be NULL. */
+SAS_API sas_status sas_decode_combine(const sas_params* p, int n_split, const float* o_part, const float* lse_part,
+                              sas_bf16* o, float* lse_o, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics
+ * ------------------------------------------------------------------------- */
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device. *code is SAS_OK when no kernel raised an error since the
+ * last read, else the first sas_status a kernel raised (SAS_ERR_TIMEOUT or
+ * SAS_ERR_DEVICE_INDEX). */
+SAS_API sas_status sas_get_device_error(void* stream, int* code);
+
+/* Static, human-readable name of a status code. */
+SAS_API const char* sas_status_string(sas_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+SAS_API int sas_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAS_H_ */

@@ -1,0 +1,268 @@
+"""Python binding of the SAS gated block-sparse attention library (B200, sm_100a).
+
+A thin ctypes layer over ``libsas_b200.so``. Every function named like a C
+entry point marshals torch tensors into device pointers and calls the C
+function. All computation runs in the library's CUDA kernels, and nothing
+here falls back to PyTorch or the CPU. Importing this package fails loudly
+when the library has not been built (``python -m learned_block_sparse_warp_b200.build``).
+
+The entry points and their contracts are those of include/sas.h:
+``sas_topk_select``, ``sas_gate_lse``, ``sas_fwd``, ``sas_bwd``
+(+ ``sas_bwd_workspace_size``), ``sas_decode``, ``sas_decode_combine``,
+``sas_get_device_error``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "SAS_GATE_LOG_SOFTMAX", "SAS_GATE_NONE", "SasError", "Params", "lib",
+    "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd", "sas_decode",
+    "sas_decode_combine", "sas_get_device_error", "sas_status_string", "sas_version",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
+
+SAS_GATE_LOG_SOFTMAX = 0
+SAS_GATE_NONE = 1
+STATUS = {0: "SAS_OK", 1: "SAS_ERR_INVALID_ARG", 2: "SAS_ERR_UNSUPPORTED", 3: "SAS_ERR_WORKSPACE",
+          4: "SAS_ERR_CUDA", 5: "SAS_ERR_TIMEOUT", 6: "SAS_ERR_DEVICE_INDEX"}
+BLOCK = 64
+
+
+class SasError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {sas_status_string(code)}")
+
+
+class sas_params(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("seq_len", ctypes.c_int), ("block", ctypes.c_int),
+        ("top_k", ctypes.c_int), ("softmax_scale", ctypes.c_float), ("gate_mode", ctypes.c_int),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m learned_block_sparse_warp_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(sas_params)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    sig = {
+        "sas_topk_select": [P, vp, vp, vp, vp, vp],
+        "sas_gate_lse": [P, vp, vp, vp, vp],
+        "sas_fwd": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "sas_bwd_workspace_size": [P, ctypes.POINTER(sz)],
+        "sas_bwd": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "sas_decode": [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp],
+        "sas_decode_combine": [P, ctypes.c_int, vp, vp, vp, vp, vp],
+        "sas_get_device_error": [vp, ctypes.POINTER(ctypes.c_int)],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    L.sas_status_string.argtypes = [ctypes.c_int]
+    L.sas_status_string.restype = ctypes.c_char_p
+    L.sas_version.argtypes = []
+    L.sas_version.restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def sas_status_string(code: int) -> str:
+    return lib.sas_status_string(int(code)).decode()
+
+
+def sas_version() -> int:
+    return int(lib.sas_version())
+
+
+@dataclass
+class Params:
+    """Mirror of ``sas_params``. ``seq_len`` is N for prefill and Lmax for decode."""
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    seq_len: int
+    top_k: int
+    block: int = BLOCK
+    softmax_scale: float = 0.0
+    gate_mode: int = SAS_GATE_LOG_SOFTMAX
+
+    @property
+    def n_blocks(self) -> int:
+        return self.seq_len // self.block
+
+    @property
+    def group(self) -> int:
+        return self.n_q_heads // self.n_kv_heads
+
+    def c(self) -> sas_params:
+        return sas_params(self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim, self.seq_len, self.block,
+                          self.top_k, float(self.softmax_scale), int(self.gate_mode))
+
+
+def _ptr(t: Optional[torch.Tensor], dtype: Optional[torch.dtype] = None, shape=None, name: str = "?"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise SasError(fn, code)
+
+
+def _shapes(p: Params, decode: bool):
+    B, Hq, Hkv, d, NB, K = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.n_blocks, p.top_k
+    if decode:
+        return dict(s=(B, Hkv, NB), idx=(B, Hkv, K), lse_s=(B, Hkv))
+    return dict(s=(B, Hkv, NB, NB), idx=(B, Hkv, NB, K), lse_s=(B, Hkv, NB), q=(B, Hq, p.seq_len, d),
+                kv=(B, Hkv, p.seq_len, d), lse_o=(B, Hq, p.seq_len))
+
+
+bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+
+
+def sas_topk_select(p: Params, s: torch.Tensor, idx: torch.Tensor, lse_s: Optional[torch.Tensor] = None,
+                    cache_len: Optional[torch.Tensor] = None, stream=None) -> None:
+    sh = _shapes(p, cache_len is not None)
+    _check("sas_topk_select", lib.sas_topk_select(
+        ctypes.byref(p.c()), _ptr(s, f32, sh["s"], "s"), _ptr(cache_len, i32, (p.batch,), "cache_len"),
+        _ptr(idx, i32, sh["idx"], "idx"), _ptr(lse_s, f32, sh["lse_s"], "lse_s"), _stream(stream)))
+
+
+def sas_gate_lse(p: Params, s: torch.Tensor, lse_s: torch.Tensor, cache_len: Optional[torch.Tensor] = None,
+                 stream=None) -> None:
+    sh = _shapes(p, cache_len is not None)
+    _check("sas_gate_lse", lib.sas_gate_lse(
+        ctypes.byref(p.c()), _ptr(s, f32, sh["s"], "s"), _ptr(cache_len, i32, (p.batch,), "cache_len"),
+        _ptr(lse_s, f32, sh["lse_s"], "lse_s"), _stream(stream)))
+
+
+def sas_fwd(p: Params, q, k, v, s, idx, lse_s, o, lse_o=None, stream=None) -> None:
+    sh = _shapes(p, False)
+    _check("sas_fwd", lib.sas_fwd(
+        ctypes.byref(p.c()), _ptr(q, bf16, sh["q"], "q"), _ptr(k, bf16, sh["kv"], "k"), _ptr(v, bf16, sh["kv"], "v"),
+        _ptr(s, f32, sh["s"], "s"), _ptr(idx, i32, sh["idx"], "idx"), _ptr(lse_s, f32, sh["lse_s"], "lse_s"),
+        _ptr(o, bf16, sh["q"], "o"), _ptr(lse_o, f32, sh["lse_o"], "lse_o"), _stream(stream)))
+
+
+def sas_bwd_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t(0)
+    _check("sas_bwd_workspace_size", lib.sas_bwd_workspace_size(ctypes.byref(p.c()), ctypes.byref(n)))
+    return int(n.value)
+
+
+def sas_bwd(p: Params, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws: torch.Tensor, stream=None) -> None:
+    sh = _shapes(p, False)
+    _check("sas_bwd", lib.sas_bwd(
+        ctypes.byref(p.c()), _ptr(q, bf16, sh["q"], "q"), _ptr(k, bf16, sh["kv"], "k"), _ptr(v, bf16, sh["kv"], "v"),
+        _ptr(o, bf16, sh["q"], "o"), _ptr(dO, bf16, sh["q"], "dO"), _ptr(s, f32, sh["s"], "s"),
+        _ptr(idx, i32, sh["idx"], "idx"), _ptr(lse_s, f32, sh["lse_s"], "lse_s"),
+        _ptr(lse_o, f32, sh["lse_o"], "lse_o"), _ptr(dq, bf16, sh["q"], "dq"), _ptr(dk, bf16, sh["kv"], "dk"),
+        _ptr(dv, bf16, sh["kv"], "dv"), _ptr(ds, f32, sh["s"], "ds"), _ptr(ws, None, None, "ws"),
+        ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)))
+
+
+def sas_decode(p: Params, q, kc, vc, cache_len, s, idx, lse_s, n_split: int, o_part, lse_part, stream=None) -> None:
+    B, Hq, Hkv, d = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim
+    sh = _shapes(p, True)
+    _check("sas_decode", lib.sas_decode(
+        ctypes.byref(p.c()), _ptr(q, bf16, (B, Hq, d), "q"), _ptr(kc, bf16, (B, Hkv, p.seq_len, d), "kc"),
+        _ptr(vc, bf16, (B, Hkv, p.seq_len, d), "vc"), _ptr(cache_len, i32, (B,), "cache_len"),
+        _ptr(s, f32, sh["s"], "s"), _ptr(idx, i32, sh["idx"], "idx"), _ptr(lse_s, f32, sh["lse_s"], "lse_s"),
+        int(n_split), _ptr(o_part, f32, (B, Hq, n_split, d), "o_part"),
+        _ptr(lse_part, f32, (B, Hq, n_split), "lse_part"), _stream(stream)))
+
+
+def sas_decode_combine(p: Params, n_split: int, o_part, lse_part, o, lse_o=None, stream=None) -> None:
+    B, Hq, d = p.batch, p.n_q_heads, p.head_dim
+    _check("sas_decode_combine", lib.sas_decode_combine(
+        ctypes.byref(p.c()), int(n_split), _ptr(o_part, f32, (B, Hq, n_split, d), "o_part"),
+        _ptr(lse_part, f32, (B, Hq, n_split), "lse_part"), _ptr(o, bf16, (B, Hq, d), "o"),
+        _ptr(lse_o, f32, (B, Hq), "lse_o"), _stream(stream)))
+
+
+def sas_get_device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check("sas_get_device_error", lib.sas_get_device_error(_stream(stream), ctypes.byref(code)))
+    return int(code.value)
+
+
+# ---------------------------------------------------------------------------
+# Allocation helpers (device memory comes from PyTorch)
+# ---------------------------------------------------------------------------
+def empty_prefill_outputs(p: Params, device="cuda", backward: bool = True) -> dict:
+    B, Hq, Hkv, N, d, NB, K = p.batch, p.n_q_heads, p.n_kv_heads, p.seq_len, p.head_dim, p.n_blocks, p.top_k
+    out = dict(
+        idx=torch.empty((B, Hkv, NB, K), dtype=i32, device=device),
+        lse_s=torch.empty((B, Hkv, NB), dtype=f32, device=device),
+        o=torch.empty((B, Hq, N, d), dtype=bf16, device=device),
+        lse_o=torch.empty((B, Hq, N), dtype=f32, device=device),
+    )
+    if backward:
+        out.update(
+            dq=torch.empty((B, Hq, N, d), dtype=bf16, device=device),
+            dk=torch.empty((B, Hkv, N, d), dtype=bf16, device=device),
+            dv=torch.empty((B, Hkv, N, d), dtype=bf16, device=device),
+            ds=torch.empty((B, Hkv, NB, NB), dtype=f32, device=device),
+            ws=torch.empty((sas_bwd_workspace_size(p),), dtype=torch.uint8, device=device),
+        )
+    return out
+
+
+def empty_decode_outputs(p: Params, n_split: int, device="cuda") -> dict:
+    B, Hq, Hkv, d, K = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.top_k
+    return dict(
+        idx=torch.empty((B, Hkv, K), dtype=i32, device=device),
+        lse_s=torch.empty((B, Hkv), dtype=f32, device=device),
+        o_part=torch.empty((B, Hq, n_split, d), dtype=f32, device=device),
+        lse_part=torch.empty((B, Hq, n_split), dtype=f32, device=device),
+        o=torch.empty((B, Hq, d), dtype=bf16, device=device),
+        lse_o=torch.empty((B, Hq), dtype=f32, device=device),
+    )
+
+
+def prefill_step(p: Params, q, k, v, s, dO, out: dict, backward: bool = True, stream=None) -> None:
+    """One pass of the training hot path: select + LSE, forward, backward with ds."""
+    sas_topk_select(p, s, out["idx"], out["lse_s"], stream=stream)
+    sas_fwd(p, q, k, v, s, out["idx"], out["lse_s"], out["o"], out["lse_o"], stream=stream)
+    if backward:
+        sas_bwd(p, q, k, v, out["o"], dO, s, out["idx"], out["lse_s"], out["lse_o"], out["dq"], out["dk"], out["dv"],
+                out["ds"], out["ws"], stream=stream)
+
+
+def decode_step(p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, stream=None) -> None:
+    """One decode step: Top-K select (decode form), split-K attention, LSE merge."""
+    sas_topk_select(p, s, out["idx"], out["lse_s"], cache_len=cache_len, stream=stream)
+    sas_decode(p, q, kc, vc, cache_len, s, out["idx"], out["lse_s"], n_split, out["o_part"], out["lse_part"],
+               stream=stream)
+    sas_decode_combine(p, n_split, out["o_part"], out["lse_part"], out["o"], out["lse_o"], stream=stream)

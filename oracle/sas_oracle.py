@@ -259,8 +259,9 @@ def backward(q, k, v, s, idx, do, block: int = 64, gate_mode: int = GATE_LOG_SOF
                     Drow = np.sum(dOb * ob, axis=1, keepdims=True)  # = Σ_j P_ij dP_ij
                     dZ = P * (dP - Drow)  # ∂/∂z through the row softmax
                     dq[b, hq, rows] += scale * (dZ @ Kst)
-                    np.add.at(dk[b, h], tok, scale * (dZ.T @ q[b, hq, rows]))
-                    np.add.at(dv[b, h], tok, P.T @ dOb)
+                    # tok holds distinct positions, so fancy-index += sums each row once
+                    dk[b, h, tok] += scale * (dZ.T @ q[b, hq, rows])
+                    dv[b, h, tok] += P.T @ dOb
                     dlam_tok += dZ.sum(axis=0)
                 if gate_mode == GATE_NONE or t == 0:
                     continue

@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library links the CUDA runtime statically and opens the driver only on
+its first CUDA call. It therefore loads on a host without a GPU. These tests
+call only what returns before any CUDA call: status strings, the version,
+the workspace size, and argument checks that reject their input. Fake device
+pointers appear only in calls that a check rejects before any launch.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import learned_block_sparse_warp_b200 as sas
+from learned_block_sparse_warp_b200 import Params, lib, sas_params
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+A = 0x7F0000000000  # aligned fake address; only ever handed to calls that reject their arguments
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"SAS_API\s+[\w\s\*]+?\b(sas_\w+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert {"sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd", "sas_bwd_workspace_size", "sas_decode",
+            "sas_decode_combine", "sas_get_device_error", "sas_status_string", "sas_version"} <= names
+    raw = ctypes.CDLL(sas.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+
+
+def test_status_strings_and_version():
+    for code, name in sas.STATUS.items():
+        assert sas.sas_status_string(code).startswith(name)
+    assert "unknown" in sas.sas_status_string(99)
+    assert sas.sas_version() >= 100
+
+
+def _p(**kw):
+    base = dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, seq_len=1024, top_k=4)
+    base.update(kw)
+    return Params(**base)
+
+
+def _fwd(p, q=A, k=A, v=A, s=A, idx=A, lse_s=A, o=A, lse_o=None):
+    c = p.c() if p is not None else None
+    return lib.sas_fwd(ctypes.byref(c) if c is not None else None, q, k, v, s, idx, lse_s, o, lse_o, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), UNSUPPORTED),
+    (dict(head_dim=256), UNSUPPORTED),
+    (dict(block=32), UNSUPPORTED),
+    (dict(seq_len=1000), INVALID),
+    (dict(seq_len=0), INVALID),
+    (dict(n_q_heads=3), INVALID),
+    (dict(top_k=0), INVALID),
+    (dict(top_k=257), INVALID),
+    (dict(batch=0), INVALID),
+    (dict(gate_mode=7), INVALID),
+    (dict(softmax_scale=-1.0), INVALID),
+    (dict(softmax_scale=float("nan")), INVALID),
+])
+def test_fwd_rejects_bad_params(kw, code):
+    assert _fwd(_p(**kw)) == code
+
+
+def test_null_params_and_pointers():
+    assert _fwd(None) == INVALID
+    assert _fwd(_p(), q=None) == INVALID
+    assert _fwd(_p(), idx=None) == INVALID
+    assert _fwd(_p(), o=None) == INVALID
+    # gated needs s and lse_s
+    assert _fwd(_p(), s=None) == INVALID
+    assert _fwd(_p(), lse_s=None) == INVALID
+
+
+def test_misaligned_pointers_rejected():
+    assert _fwd(_p(), q=A + 2) == INVALID
+    assert _fwd(_p(), lse_o=A + 4) == INVALID
+    c = _p().c()
+    assert lib.sas_topk_select(ctypes.byref(c), A + 8, None, A, None, None) == INVALID
+    assert lib.sas_topk_select(ctypes.byref(c), A, None, None, None, None) == INVALID
+    assert lib.sas_gate_lse(ctypes.byref(c), A, None, None, None) == INVALID
+
+
+def test_workspace_size_and_check():
+    p = _p(batch=2, n_q_heads=8, n_kv_heads=2, seq_len=2048, top_k=8)
+    n = sas.sas_bwd_workspace_size(p)
+    B, Hq, Hkv, N, d, NB, K = 2, 8, 2, 2048, 128, 32, 8
+    lower = 4 * (B * Hq * N * d + B * Hq * N + B * Hkv * NB * K) + 4 * (B * Hkv * NB * 2 + B * Hkv * NB * K)
+    assert lower <= n <= lower + 6 * 256
+    c = p.c()
+    args = [A] * 13
+    # too small, unaligned, or missing workspace: SAS_ERR_WORKSPACE before any launch
+    assert lib.sas_bwd(ctypes.byref(c), *args, A, n - 1, None) == WORKSPACE
+    assert lib.sas_bwd(ctypes.byref(c), *args, A + 16, n, None) == WORKSPACE
+    assert lib.sas_bwd(ctypes.byref(c), *args, None, n, None) == WORKSPACE
+    size = ctypes.c_size_t(0)
+    assert lib.sas_bwd_workspace_size(None, ctypes.byref(size)) == INVALID
+    assert lib.sas_bwd_workspace_size(ctypes.byref(c), None) == INVALID
+
+
+def test_decode_split_count_checked():
+    c = _p(top_k=4).c()
+    base = [A, A, A, A, A, A, A]
+    assert lib.sas_decode(ctypes.byref(c), *base, 0, A, A, None) == INVALID
+    assert lib.sas_decode(ctypes.byref(c), *base, 6, A, A, None) == INVALID  # > K + 1
+    assert lib.sas_decode_combine(ctypes.byref(c), 0, A, A, A, None, None) == INVALID
+    c16 = _p(n_q_heads=32, n_kv_heads=2).c()  # G = 16: no decode kernel
+    assert lib.sas_decode(ctypes.byref(c16), *base, 2, A, A, None) == UNSUPPORTED
+
+
+def test_params_struct_layout():
+    assert ctypes.sizeof(sas_params) == 9 * 4
+    assert [f[0] for f in sas_params._fields_] == ["batch", "n_q_heads", "n_kv_heads", "head_dim", "seq_len",
+                                                    "block", "top_k", "softmax_scale", "gate_mode"]
+    hdr = open(os.path.join(ROOT, "include", "sas.h")).read()
+    body = hdr[hdr.index("typedef struct {"):hdr.index("} sas_params;")]
+    assert re.findall(r"(?:int|float)\s+(\w+);", body) == [f[0] for f in sas_params._fields_]
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    p = _p(seq_len=128, top_k=1, n_q_heads=2, n_kv_heads=2, head_dim=64)
+    s = torch.zeros(1, 2, 2, 2)
+    idx = torch.zeros(1, 2, 2, 1, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        sas.sas_topk_select(p, s, idx)

@@ -1,0 +1,54 @@
+"""GPU parity: backward dq/dk/dv and the score gradient ds against the fp64 oracle."""
+import numpy as np
+import pytest
+
+import oracle.sas_oracle as O
+from synth import workloads as W
+from tests.parity_util import TOL_REL, assert_idx_equal, rel_fro
+from tests.test_gpu_fwd import run_prefill
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("tiny", 1, 2, 2, 64, 1024, 4),
+    ("gqa4_d128", 1, 8, 2, 128, 1024, 4),
+    ("gqa5_d128", 1, 10, 2, 128, 768, 3),
+    ("dense_k", 1, 2, 1, 64, 512, 16),
+    ("one_block", 2, 2, 2, 128, 64, 4),
+    ("k1_batch2", 2, 4, 4, 64, 640, 1),
+]
+
+
+@pytest.mark.parametrize("gate", [O.GATE_LOG_SOFTMAX, O.GATE_NONE])
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_bwd_parity(case, gate):
+    name, B, Hq, Hkv, d, N, K = case
+    w = W.custom(name, batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=N, top_k=K, seed=200 + len(name))
+    x, r, err = run_prefill(w, gate, backward=True)
+    assert err == 0
+    ref_idx, _ = O.prefill_select(x["s"].astype(np.float64), K)
+    assert_idx_equal(r["idx"], ref_idx)
+    dq, dk, dv, ds, _ = O.backward(x["q"], x["k"], x["v"], x["s"], ref_idx, x["do"], gate_mode=gate)
+    errs = {n: rel_fro(r[n], ref) for n, ref in (("dq", dq), ("dk", dk), ("dv", dv))}
+    assert all(e < TOL_REL for e in errs.values()), errs
+    if gate == O.GATE_NONE:
+        assert np.all(r["ds"] == 0)
+    elif N > 64:
+        e = rel_fro(r["ds"], ds)
+        assert e < TOL_REL, e
+        # entries at or above the diagonal are exactly zero
+        NB = N // 64
+        iu = np.triu_indices(NB)
+        assert np.all(r["ds"][..., iu[0], iu[1]] == 0)
+    else:
+        assert np.all(r["ds"] == 0)
+
+
+def test_bwd_tiny_workload_exact_config():
+    w = W.WORKLOADS["tiny"]
+    x, r, err = run_prefill(w, O.GATE_LOG_SOFTMAX, backward=True)
+    assert err == 0
+    ref_idx, _ = O.prefill_select(x["s"].astype(np.float64), w.top_k)
+    dq, dk, dv, ds, _ = O.backward(x["q"], x["k"], x["v"], x["s"], ref_idx, x["do"])
+    for n, ref in (("dq", dq), ("dk", dk), ("dv", dv), ("ds", ds)):
+        assert rel_fro(r[n], ref) < TOL_REL, (n, rel_fro(r[n], ref))

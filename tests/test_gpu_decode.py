@@ -1,0 +1,74 @@
+"""GPU parity: split-K decode partials and their LSE merge against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.sas_oracle as O
+from tests.parity_util import TOL_L, TOL_O, assert_idx_equal, bf16_dev, f32_dev, host, max_abs
+from synth.workloads import bf16_round
+
+pytestmark = pytest.mark.gpu
+
+
+def _sas():
+    import learned_block_sparse_warp_b200 as sas
+    return sas
+
+
+def _case(B, Hq, Hkv, d, Lmax, seed):
+    g = np.random.default_rng(seed)
+    q = bf16_round(g.standard_normal((B, Hq, d)).astype(np.float32))
+    kc = bf16_round(g.standard_normal((B, Hkv, Lmax, d)).astype(np.float32))
+    vc = bf16_round(g.standard_normal((B, Hkv, Lmax, d)).astype(np.float32))
+    s = (g.standard_normal((B, Hkv, Lmax // 64)) * np.sqrt(2)).astype(np.float32)
+    return q, kc, vc, s
+
+
+@pytest.mark.parametrize("gate", [O.GATE_NONE, O.GATE_LOG_SOFTMAX])
+@pytest.mark.parametrize("B,Hq,Hkv,d,Lmax,K,n_split,lens", [
+    (4, 32, 8, 128, 2048, 16, 17, [2048, 1, 1000, 1999]),
+    (3, 8, 8, 64, 1024, 4, 2, [64, 65, 1024]),
+    (2, 10, 2, 128, 4096, 8, 3, [4096, 4033]),
+    (2, 16, 2, 128, 1024, 32, 33, [1024, 130]),   # K above the history: every block, G = 8
+    (1, 4, 1, 64, 512, 2, 1, [300]),
+])
+def test_decode_parity(B, Hq, Hkv, d, Lmax, K, n_split, lens, gate):
+    sas = _sas()
+    q, kc, vc, s = _case(B, Hq, Hkv, d, Lmax, seed=B * 31 + K)
+    cl = np.array(lens, dtype=np.int32)
+    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=Lmax, top_k=K, gate_mode=gate)
+    out = sas.empty_decode_outputs(p, n_split)
+    sas.decode_step(p, bf16_dev(q), bf16_dev(kc), bf16_dev(vc), torch.from_numpy(cl).cuda(), f32_dev(s), n_split, out)
+    torch.cuda.synchronize()
+    assert sas.sas_get_device_error() == 0
+    ref = O.decode(q, kc, vc, cl, s.astype(np.float64), K, gate_mode=gate, n_split=n_split)
+    assert_idx_equal(out["idx"].cpu().numpy(), ref["idx"])
+    # split partials: same chunking of the block list on both sides
+    lp = host(out["lse_part"])
+    fin = np.isfinite(ref["lse_part"])
+    assert np.array_equal(np.isfinite(lp), fin)
+    assert max_abs(lp[fin], ref["lse_part"][fin]) < TOL_L
+    assert max_abs(host(out["o_part"]), ref["o_part"]) < TOL_O
+    assert max_abs(host(out["o"]), ref["o"]) < TOL_O
+    assert max_abs(host(out["lse_o"]), ref["lse"]) < TOL_L
+
+
+def test_combine_on_oracle_partials():
+    """The merge kernel alone, fed partials the oracle computed (including empty splits)."""
+    sas = _sas()
+    B, Hq, d, ns = 3, 4, 128, 5
+    g = np.random.default_rng(9)
+    o_part = g.standard_normal((B, Hq, ns, d))
+    lse_part = g.standard_normal((B, Hq, ns)) * 3
+    lse_part[0, 1, 2] = -np.inf
+    lse_part[2, 3, :] = -np.inf
+    lse_part[2, 3, 4] = 0.5
+    o_part[lse_part == -np.inf] = 0.0
+    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hq, head_dim=d, seq_len=1024, top_k=8)
+    o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    sas.sas_decode_combine(p, ns, f32_dev(o_part), f32_dev(lse_part), o, lse)
+    torch.cuda.synchronize()
+    ref_o, ref_lse = O.decode_combine(o_part, lse_part)
+    assert max_abs(host(o), ref_o) < TOL_O
+    assert max_abs(host(lse), ref_lse) < 1e-5
