@@ -204,6 +204,50 @@ SAS_API sas_status sas_decode_combine(const sas_params* p, int n_split, const fl
                               sas_bf16* o, float* lse_o, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Decode step that allocates nothing. The paper has no counterpart to this
+ * entry point; it exists for callers of this library that cannot allocate.
+ * ------------------------------------------------------------------------- */
+
+/* Size of the library's fixed decode scratch, on every GPU that loads it. */
+#define SAS_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+
+/* The whole decode step in one call: the decode form of sas_topk_select, then
+ * sas_decode with n_split = K + 1 (one block per split), then
+ * sas_decode_combine. The caller passes the inputs and the outputs only. The
+ * index lists, gate normalisers and split partials between the kernels live in
+ * a fixed device array inside the library, so the call allocates nothing.
+ *
+ * Who needs it: callers that cannot call cudaMalloc. cudaMalloc synchronises
+ * the device, which a serving loop with a per-step latency budget cannot
+ * afford. A plugin inside a host framework whose caching allocator already
+ * holds most of HBM would see cudaMalloc fail or fragment memory behind the
+ * framework's back. A plain C caller may have no device allocator at all.
+ *
+ * Arguments: q, kc, vc, cache_len and s as in sas_decode (s is always
+ * required, it drives the selection). o bf16 [B, Hq, d] and lse_o fp32
+ * [B, Hq] (may be NULL) as in sas_decode_combine.
+ *
+ * Limits and behaviour:
+ *  - The scratch holds B·Hkv·K int32 indices, B·Hkv fp32 normalisers and
+ *    B·Hq·(K+1)·(d+1) fp32 partials, each region rounded up to 256 bytes.
+ *    Sizes beyond SAS_NOALLOC_SCRATCH_BYTES return SAS_ERR_WORKSPACE before
+ *    any launch. For example, 16 sequences × 32 query heads × K = 16 × d = 128
+ *    need about 4.5 MB.
+ *  - The array is a file-scope device variable: every GPU that loads the
+ *    library holds these 16 MiB until the process exits.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current). Make that first call
+ *    before any stream capture on that device.
+ *  - Every call shares the one array per device. Calls that overlap on the
+ *    GPU (other streams, other host threads) race on it; the caller must
+ *    order them. Each call writes all the scratch it reads, so nothing needs
+ *    clearing between calls.
+ *  - No cudaMalloc, cudaFree or allocating library routine is called. */
+SAS_API sas_status sas_decode_noalloc(const sas_params* p, const sas_bf16* q, const sas_bf16* kc, const sas_bf16* vc,
+                                      const int32_t* cache_len, const float* s, sas_bf16* o, float* lse_o,
+                                      void* stream);
+
+/* ---------------------------------------------------------------------------
  * Diagnostics
  * ------------------------------------------------------------------------- */
 

@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "SAS_GATE_LOG_SOFTMAX", "SAS_GATE_NONE", "SasError", "Params", "lib",
     "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd", "sas_decode",
-    "sas_decode_combine", "sas_get_device_error", "sas_status_string", "sas_version",
+    "sas_decode_combine", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string", "sas_version",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
@@ -64,6 +64,7 @@ def _load() -> ctypes.CDLL:
         "sas_decode": [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp],
         "sas_decode_combine": [P, ctypes.c_int, vp, vp, vp, vp, vp],
         "sas_get_device_error": [vp, ctypes.POINTER(ctypes.c_int)],
+        "sas_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -209,6 +210,16 @@ def sas_decode_combine(p: Params, n_split: int, o_part, lse_part, o, lse_o=None,
         ctypes.byref(p.c()), int(n_split), _ptr(o_part, f32, (B, Hq, n_split, d), "o_part"),
         _ptr(lse_part, f32, (B, Hq, n_split), "lse_part"), _ptr(o, bf16, (B, Hq, d), "o"),
         _ptr(lse_o, f32, (B, Hq), "lse_o"), _stream(stream)))
+
+
+def sas_decode_noalloc(p: Params, q, kc, vc, cache_len, s, o, lse_o=None, stream=None) -> None:
+    """Whole decode step with the library's fixed device scratch (see include/sas.h)."""
+    B, Hq, Hkv, d = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim
+    _check("sas_decode_noalloc", lib.sas_decode_noalloc(
+        ctypes.byref(p.c()), _ptr(q, bf16, (B, Hq, d), "q"), _ptr(kc, bf16, (B, Hkv, p.seq_len, d), "kc"),
+        _ptr(vc, bf16, (B, Hkv, p.seq_len, d), "vc"), _ptr(cache_len, i32, (B,), "cache_len"),
+        _ptr(s, f32, (B, Hkv, p.n_blocks), "s"), _ptr(o, bf16, (B, Hq, d), "o"), _ptr(lse_o, f32, (B, Hq), "lse_o"),
+        _stream(stream)))
 
 
 def sas_get_device_error(stream=None) -> int:

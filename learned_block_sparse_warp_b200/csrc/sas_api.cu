@@ -89,6 +89,13 @@ sas_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SAS_OK : SAS_ERR
 
 }  // namespace
 
+namespace sas {
+// Parameter checks and the device error word, shared with the other
+// entry-point files of the library.
+sas_status check_params(const sas_params* p, Shape* sh) { return make_shape(p, sh); }
+int* error_word() { return device_error_word(); }
+}  // namespace sas
+
 extern "C" {
 
 int sas_version(void) { return 100; }
