@@ -222,104 +222,136 @@ def run_gpu(args, rank, world, local_rank):
         return float(t.item())
 
     stream = torch.cuda.Stream(device=dev)
-    w = W.WORKLOADS[TRAIN]
-    p = sas.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
-                   seq_len=w.seq_len, top_k=w.top_k, gate_mode=sas.SAS_GATE_LOG_SOFTMAX)
-    x = prefill_to_device(w, device=dev)
-    out = sas.empty_prefill_outputs(p, device=dev)
-    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
-
-    def step(q, k, v, s, dO, o):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        ev[0].record(stream)
-        sas.sas_topk_select(p, s, o["idx"], o["lse_s"], stream=stream)
-        ev[1].record(stream)
-        sas.sas_fwd(p, q, k, v, s, o["idx"], o["lse_s"], o["o"], o["lse_o"], stream=stream)
-        ev[2].record(stream)
-        sas.sas_bwd(p, q, k, v, o["o"], dO, s, o["idx"], o["lse_s"], o["lse_o"], o["dq"], o["dk"], o["dv"],
-                    o["ds"], o["ws"], stream=stream)
-        ev[3].record(stream)
-        return ev
-
-    evs = []
-    with ClockSampler(local_rank) as clk:
-        clk.wait_first()
-        with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                step(x["q"], x["k"], x["v"], x["s"], x["do"], out)
-        torch.cuda.synchronize()
-        if sas.sas_get_device_error(stream) != 0:
-            raise RuntimeError("device error during warm-up")
-        barrier()
-        torch.cuda.synchronize()
-        clk.mark("t_begin")
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for _ in range(args.steps):
-            evs.append(step(x["q"], x["k"], x["v"], x["s"], x["do"], out))
-        t_end.record(stream)
-        torch.cuda.synchronize()
-        clk.mark("t_end")
-        time.sleep(0.25)
-    barrier()
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
-    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-
-    F = fwd_flops(w.n_q_heads, w.head_dim, w.n_blocks, w.top_k, batch=w.batch)
-    step_flops = 3.5 * F
-    ms_per_step = total_ms / args.steps
-    value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
     pk = peaks()
+    line = {}
 
-    # end to end through the public API: pinned host inputs in, every output back to pinned host memory
-    e2e = None
-    if not args.no_e2e:
-        h_in = {k_: t.cpu().pin_memory() for k_, t in x.items()}
-        d_in = {k_: torch.empty_like(t) for k_, t in x.items()}
-        outs = ["o", "lse_o", "dq", "dk", "dv", "ds"]
-        h_out = {k_: torch.empty(out[k_].shape, dtype=out[k_].dtype, pin_memory=True) for k_ in outs}
-        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
-        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    # ---------------- training step: select + LSE, forward, backward with ds ----------------
+    if args.only in ("all", "train"):
+        w = W.WORKLOADS[TRAIN]
+        p = sas.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
+                       seq_len=w.seq_len, top_k=w.top_k, gate_mode=sas.SAS_GATE_LOG_SOFTMAX)
+        x = prefill_to_device(w, device=dev)
+        out = sas.empty_prefill_outputs(p, device=dev)
+        in_bytes = sum(t.numel() * t.element_size() for t in x.values())
 
-        def e2e_step():
+        def step(q, k, v, s, dO, o):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
+            sas.sas_topk_select(p, s, o["idx"], o["lse_s"], stream=stream)
+            ev[1].record(stream)
+            sas.sas_fwd(p, q, k, v, s, o["idx"], o["lse_s"], o["o"], o["lse_o"], stream=stream)
+            ev[2].record(stream)
+            sas.sas_bwd(p, q, k, v, o["o"], dO, s, o["idx"], o["lse_s"], o["lse_o"], o["dq"], o["dk"], o["dv"],
+                        o["ds"], o["ws"], stream=stream)
+            ev[3].record(stream)
+            return ev
+
+        evs = []
+        with ClockSampler(local_rank) as clk:
+            clk.wait_first()
             with torch.cuda.stream(stream):
-                for k_ in d_in:
-                    d_in[k_].copy_(h_in[k_], non_blocking=True)
-                step(d_in["q"], d_in["k"], d_in["v"], d_in["s"], d_in["do"], out)
-                for k_ in outs:
-                    h_out[k_].copy_(out[k_], non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        n_e2e = max(1, min(args.steps, 3))
+                for _ in range(args.warmup):
+                    step(x["q"], x["k"], x["v"], x["s"], x["do"], out)
+            torch.cuda.synchronize()
+            if sas.sas_get_device_error(stream) != 0:
+                raise RuntimeError("device error during warm-up")
+            barrier()
+            torch.cuda.synchronize()
+            clk.mark("t_begin")
+            t_start = torch.cuda.Event(enable_timing=True)
+            t_end = torch.cuda.Event(enable_timing=True)
+            t_start.record(stream)
+            for _ in range(args.steps):
+                evs.append(step(x["q"], x["k"], x["v"], x["s"], x["do"], out))
+            t_end.record(stream)
+            torch.cuda.synchronize()
+            clk.mark("t_end")
+            time.sleep(0.25)
         barrier()
-        torch.cuda.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(a.elapsed_time(b)) / n_e2e
-        e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e}
-        del h_in, d_in, h_out
+        total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+        sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+        fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+        if sas.sas_get_device_error(stream) != 0:
+            raise RuntimeError("device error during the timed steps")
 
-    # decode workload: split-K + merge, L2 flushed before every timed step
-    dec = None
-    if not args.no_decode:
-        del x
+        F = fwd_flops(w.n_q_heads, w.head_dim, w.n_blocks, w.top_k, batch=w.batch)
+        step_flops = 3.5 * F
+
+        # end to end through the public API: pinned host inputs in, every output back to pinned host memory
+        e2e = None
+        if not args.no_e2e:
+            h_in = {k_: t.cpu().pin_memory() for k_, t in x.items()}
+            d_in = {k_: torch.empty_like(t) for k_, t in x.items()}
+            outs = ["o", "lse_o", "dq", "dk", "dv", "ds"]
+            h_out = {k_: torch.empty(out[k_].shape, dtype=out[k_].dtype, pin_memory=True) for k_ in outs}
+            h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+            d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+            def e2e_step():
+                with torch.cuda.stream(stream):
+                    for k_ in d_in:
+                        d_in[k_].copy_(h_in[k_], non_blocking=True)
+                    step(d_in["q"], d_in["k"], d_in["v"], d_in["s"], d_in["do"], out)
+                    for k_ in outs:
+                        h_out[k_].copy_(out[k_], non_blocking=True)
+
+            e2e_step()
+            torch.cuda.synchronize()
+            n_e2e = max(1, min(args.steps, 3))
+            barrier()
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            b.record(stream)
+            torch.cuda.synchronize()
+            e2e_ms = max_over_ranks(a.elapsed_time(b)) / n_e2e
+            e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e}
+            del h_in, d_in, h_out
+
+        bwd_flops = 2.5 * F
+        achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
+        line.update({
+            "metric": METRIC, "value": world * step_flops * args.steps / (total_ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": TRAIN, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                       "head_dim": w.head_dim, "seq_len": w.seq_len, "block": w.block, "top_k": w.top_k,
+                       "gate": "log_softmax (training form)", "flops_per_step": step_flops,
+                       "parallelism": f"dp{world} (independent replicas)",
+                       "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > 126 MB L2 (no flush)"},
+            "breakdown_ms": {"select": sel_ms, "fwd": fwd_ms, "bwd": bwd_ms},
+            "fwd_tflops": F / (fwd_ms * 1e-3) / 1e12,
+            "bwd_tflops": achieved,
+            "roofline": {"bound": "tensor",
+                         "kernel": "sas_bwd call (bwd_main_kernel + prep/reverse-index/epilogue)",
+                         "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_sustained"], "peak_source": pk["source"] + " sustained bf16",
+                         "traffic": traffic_record("bwd_main", ["learned_block_sparse_warp_b200/csrc/bwd_mma.cu"])},
+            "e2e": e2e,
+            "gpu_launches": args.steps * 9,
+            "clocks": clk.summary(),
+        })
+        del x, out
+        torch.cuda.empty_cache()
+
+    # ---------------- decode: select, split-K, merge; L2 flushed before every timed step ----------------
+    if args.only in ("all", "decode") and not args.no_decode:
         wd = W.WORKLOADS[DECODE]
         pd = sas.Params(batch=wd.batch, n_q_heads=wd.n_q_heads, n_kv_heads=wd.n_kv_heads, head_dim=wd.head_dim,
                         seq_len=wd.seq_len, top_k=wd.top_k, gate_mode=sas.SAS_GATE_NONE)
         xd = decode_to_device(wd, device=dev)
-        n_split = wd.top_k + 1
+        n_split = args.n_split if args.n_split > 0 else wd.top_k + 1
         od = sas.empty_decode_outputs(pd, n_split, device=dev)
-        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        # a read-only sweep of 2x the L2 evicts the previous step's lines without leaving dirty ones,
+        # whose write-back would otherwise land inside the next timed step
+        flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        flush_sink = torch.empty((), dtype=torch.float32, device=dev)
 
         def dstep():
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -339,7 +371,7 @@ def run_gpu(args, rank, world, local_rank):
             for _ in range(max(3, args.warmup)):
                 dstep()
             for _ in range(n_dec):
-                flush.zero_()
+                torch.sum(flush, dim=0, out=flush_sink)
                 dev_evs.append(dstep())
         torch.cuda.synchronize()
         step_ms = statistics.median(e[0].elapsed_time(e[3]) for e in dev_evs)
@@ -349,43 +381,20 @@ def run_gpu(args, rank, world, local_rank):
         step_ms = max_over_ranks(step_ms)
         kv = decode_kv_bytes(wd, xd["cache_len"].cpu().numpy())
         gbs = kv / (split_ms * 1e-3) / 1e9
-        dec = {"workload": DECODE, "tok_per_s": world * wd.batch / (step_ms * 1e-3), "ms_per_step": step_ms,
-               "select_ms": sel_d_ms, "split_ms": split_ms, "combine_ms": comb_ms, "n_split": n_split,
-               "gate": "none (inference form)", "l2": "flushed (512 MB write) before every step",
-               "roofline": {"bound": "hbm", "kernel": "decode_split_kernel (sas_decode)", "achieved": gbs,
-                            "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
-                            "algorithmic_bytes": kv,
-                            "traffic": traffic_record("decode_split", ["learned_block_sparse_warp_b200/csrc/decode.cu"])},
-               "gpu_launches_per_step": 3}
+        line["decode"] = {
+            "workload": DECODE, "tok_per_s": world * wd.batch / (step_ms * 1e-3), "ms_per_step": step_ms,
+            "select_ms": sel_d_ms, "split_ms": split_ms, "combine_ms": comb_ms, "n_split": n_split,
+            "gate": "none (inference form)", "l2": "flushed (252 MB read) before every step",
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel (sas_decode)", "achieved": gbs,
+                         "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"], "algorithmic_bytes": kv,
+                         "traffic": traffic_record("decode_split",
+                                                   ["learned_block_sparse_warp_b200/csrc/decode.cu"])},
+            "gpu_launches_per_step": 3}
         if sas.sas_get_device_error(stream) != 0:
             raise RuntimeError("device error during decode")
 
-    bwd_flops = 2.5 * F
-    achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": TRAIN, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
-                   "head_dim": w.head_dim, "seq_len": w.seq_len, "block": w.block, "top_k": w.top_k,
-                   "gate": "log_softmax (training form)", "flops_per_step": step_flops,
-                   "parallelism": f"dp{world} (independent replicas)",
-                   "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > 126 MB L2 (no flush)"},
-        "breakdown_ms": {"select": sel_ms, "fwd": fwd_ms, "bwd": bwd_ms},
-        "fwd_tflops": F / (fwd_ms * 1e-3) / 1e12,
-        "bwd_tflops": achieved,
-        "roofline": {"bound": "tensor", "kernel": "sas_bwd call (bwd_main_kernel + prep/reverse-index/epilogue)",
-                     "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_sustained"], "peak_source": pk["source"] + " sustained bf16",
-                     "traffic": traffic_record("bwd_main", ["learned_block_sparse_warp_b200/csrc/bwd_mma.cu"])},
-        "e2e": e2e,
-        "gpu_launches": args.steps * 9,
-        "clocks": clk.summary(),
-    }
-    if dec is not None:
-        line["decode"] = dec
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_baseline(w, budget_s=args.cpu_budget)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only in ("all", "train"):
+        line["cpu_baseline"] = oracle_baseline(W.WORKLOADS[TRAIN], budget_s=args.cpu_budget)
     if dist is not None:
         dist.destroy_process_group()
     return line
@@ -425,6 +434,9 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sas", "reference"], default="sas")
+    ap.add_argument("--only", choices=["all", "train", "decode"], default="all",
+                    help="run only one workload (for profiling); the JSON line needs 'all'")
+    ap.add_argument("--n-split", type=int, default=0, help="decode splits (0: K + 1)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -26,40 +26,6 @@ __device__ __forceinline__ void load_tile_async(uint32_t s_base, const uint16_t*
   }
 }
 
-// Builds the ordered block list [t, I_t...] of one query block in shared
-// memory with each block's log2-domain gate. Run by one warp.
-__device__ __forceinline__ void build_block_list(const int32_t* __restrict__ idx_row, int K, int t,
-                                                 const float* __restrict__ s_row, float lse_t, int gated,
-                                                 int* list_s, float* lam_s, int* nlist_s, int* err) {
-  const int lane = threadIdx.x & 31;
-  const int n = min(K, t);
-  int cnt = 0;
-  bool stop = false;
-  for (int base = 0; base < n && !stop; base += 32) {
-    const int k = base + lane;
-    const int m = (k < n) ? idx_row[k] : -1;
-    const bool end = (k < n) && m < 0;
-    const bool bad = (k < n) && m >= t;
-    if (bad) raise_error(err, SAS_ERR_DEVICE_INDEX);
-    const unsigned end_mask = __ballot_sync(0xffffffffu, end);
-    const int first_end = end_mask ? __ffs(end_mask) - 1 : 32;
-    const bool ok = (k < n) && !bad && m >= 0 && lane < first_end;
-    const unsigned ok_mask = __ballot_sync(0xffffffffu, ok);
-    if (ok) {
-      const int pos = 1 + cnt + __popc(ok_mask & ((1u << lane) - 1u));
-      list_s[pos] = m;
-      lam_s[pos] = gated ? (s_row[m] - lse_t) * kLog2e : 0.f;
-    }
-    cnt += __popc(ok_mask);
-    stop = end_mask != 0;
-  }
-  if (lane == 0) {
-    list_s[0] = t;
-    lam_s[0] = 0.f;
-    *nlist_s = 1 + cnt;
-  }
-}
-
 template <int D>
 __global__ void __launch_bounds__(128) fwd_mma_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                                                       const uint16_t* __restrict__ v, const float* __restrict__ s,

@@ -1,0 +1,387 @@
+// Gated block-sparse attention forward on the Blackwell tensor cores.
+//
+// SAS explainer (ta-paperlens), section 仕組み, Eq. (9):
+//   o = softmax(q K_Sᵀ + log g_S) V_S,  S = B0 ∪ ⋃_{m∈I} B_m,
+// with log g_m = s_m − LSE(s) (SAS summary, onedev.kr, section 무엇과 다른가)
+// on every logit of history block m and 0 on the causally masked current
+// block B0.
+//
+// One CTA owns one (batch, KV head, query block) and up to four query heads
+// of the group. That is 256 rows, packed as two M = 128 tiles of two heads
+// each, so every gathered K/V block serves four heads (GQA packing). Roles:
+//   warp 0       builds the block list [t, I_t...], then issues TMA loads:
+//                the Q rows once, then the selected K/V blocks two at a time
+//                (N = 128) into a 2-stage shared-memory ring. Blocks are
+//                gathered by index with no copy in HBM.
+//   warp 1       allocates 512 TMEM columns and issues every tcgen05.mma:
+//                S_r = Q_r Kᵀ (SS, fp32 in TMEM), then O_r += P_r V (TS:
+//                P_r read from TMEM).
+//   warps 4-7    softmax of tile 0; warps 8-11 softmax of tile 1. Each thread
+//                owns one row: it reads S from TMEM, adds the block's
+//                log-gate (one scalar per 64 columns), masks the current
+//                block causally, updates the row max and sum, and writes
+//                bf16 P back over the consumed S columns. O is rescaled in
+//                TMEM only when the row max grows by more than 2^8, so the
+//                result is exact and rescales are rare.
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// Every mbarrier wait is bounded and raises SAS_ERR_TIMEOUT instead of hanging.
+#include <mutex>
+
+#include "sm100.cuh"
+
+namespace sas {
+
+namespace fsm {
+constexpr int kThreads = 384;
+constexpr int kStages = 2;
+constexpr int kHalf = 128 * 128;                 // one d-half of a 128-row tile: 128 rows x 128 B
+constexpr int kQBytes = 4 * kHalf;               // 2 tiles x 2 d-halves
+constexpr int kStageBytes = 4 * kHalf;           // K and V, 2 d-halves each, 128 token rows
+constexpr int kSmemBytes = kQBytes + kStages * kStageBytes + 1024;  // + room to align to 1 KB
+constexpr float kRescale = 8.0f;                 // log2 headroom before O is rescaled
+}  // namespace fsm
+
+struct FwdSm100Args {
+  const int32_t* idx;
+  const float* s;
+  const float* lse_s;
+  uint16_t* o;
+  float* lse_o;
+  int* err;
+  int B, Hq, Hkv, G, N, NB, K, gated, n_tp;
+  float scale;
+};
+
+__global__ void __launch_bounds__(fsm::kThreads, 1)
+    fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, FwdSm100Args a) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int list_s[kMaxTopK + 1];
+  __shared__ float lam_s[kMaxTopK + 1];
+  __shared__ int nlist_s;
+  __shared__ __align__(8) uint64_t bar_q, bar_full[fsm::kStages], bar_empty[fsm::kStages], bar_s[2], bar_p[2],
+      bar_o[2], bar_fin;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sQ = base, sKV = base + fsm::kQBytes;
+  const int t = a.NB - 1 - int(blockIdx.x);
+  const int h = int(blockIdx.y) / a.n_tp, tp = int(blockIdx.y) % a.n_tp;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g_first = 4 * tp;
+  const int n_heads = min(4, a.G - g_first);
+  const int n_tiles = (n_heads + 1) / 2;
+  const size_t bh = size_t(b) * a.Hkv + h;
+  volatile int* abort_flag = &abort_s;
+
+  if (threadIdx.x == 0) abort_s = 0;
+  if (warp == 0) {
+    const size_t row = bh * a.NB + t;
+    build_block_list(a.idx + row * a.K, a.K, t, a.gated ? a.s + row * a.NB : nullptr,
+                     a.gated ? a.lse_s[row] : 0.f, a.gated, list_s, lam_s, &nlist_s, a.err);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_s), 512);
+    if (lane == 0) {
+      mbar_init(smem_u32(&bar_q), 1);
+      for (int s = 0; s < fsm::kStages; ++s) {
+        mbar_init(smem_u32(&bar_full[s]), 1);
+        mbar_init(smem_u32(&bar_empty[s]), 1);
+      }
+      for (int r = 0; r < 2; ++r) {
+        mbar_init(smem_u32(&bar_s[r]), 1);
+        mbar_init(smem_u32(&bar_p[r]), 128);
+        mbar_init(smem_u32(&bar_o[r]), 1);
+      }
+      mbar_init(smem_u32(&bar_fin), 1);
+      fence_barrier_init();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  const int nl = nlist_s;
+  const int n_pairs = (nl + 1) / 2;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(smem_u32(&bar_q), uint32_t(n_heads) * 2u * 8192u);
+      for (int hh = 0; hh < n_heads; ++hh) {
+        const int r = hh >> 1, half = hh & 1;
+        const int row = int((size_t(b) * a.Hq + size_t(h) * a.G + g_first + hh) * a.N + size_t(t) * kBlock);
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d(sQ + (r * 2 + c) * fsm::kHalf + half * 8192, &tmQ, c * 64, row, smem_u32(&bar_q));
+      }
+      int issued = 0;
+      for (int p = 0; p < n_pairs; ++p) {
+        const int st = p % fsm::kStages, use = p / fsm::kStages;
+        if (!mbar_wait(smem_u32(&bar_empty[st]), (use & 1) ^ 1, abort_flag, a.err)) break;
+        const int nb = min(2, nl - 2 * p);
+        mbar_arrive_expect_tx(smem_u32(&bar_full[st]), uint32_t(nb) * 4u * 8192u);
+        const uint32_t sk = sKV + st * fsm::kStageBytes, sv = sk + 2 * fsm::kHalf;
+        for (int bb = 0; bb < nb; ++bb) {
+          const int row = int(bh * a.N + size_t(list_s[2 * p + bb]) * kBlock);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_2d(sk + c * fsm::kHalf + bb * 8192, &tmK, c * 64, row, smem_u32(&bar_full[st]));
+            tma_load_2d(sv + c * fsm::kHalf + bb * 8192, &tmV, c * 64, row, smem_u32(&bar_full[st]));
+          }
+        }
+        ++issued;
+      }
+      if (*abort_flag) {  // let the loads already in flight land before the CTA exits
+        for (int p = max(0, issued - fsm::kStages); p < issued; ++p) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(smem_u32(&bar_full[p % fsm::kStages]), (p / fsm::kStages) & 1) &&
+                 clock64() - t0 < kWaitCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS2 = idesc_bf16_f32(128, 128, 0, 0), idS1 = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
+      bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, a.err);
+      tc_fence_after();
+      for (int p = 0; ok && p < n_pairs; ++p) {
+        const int st = p % fsm::kStages, use = p / fsm::kStages;
+        if (!(ok = mbar_wait(smem_u32(&bar_full[st]), use & 1, abort_flag, a.err))) break;
+        tc_fence_after();
+        const int nb = min(2, nl - 2 * p);
+        const uint32_t sk = sKV + st * fsm::kStageBytes, sv = sk + 2 * fsm::kHalf;
+        for (int r = 0; r < n_tiles; ++r) {
+          if (p > 0) {  // PV_r(p-1) reads P_r from the columns that S_r(p) overwrites
+            if (!(ok = mbar_wait(smem_u32(&bar_o[r]), (p - 1) & 1, abort_flag, a.err))) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int c = k >> 2, kk = k & 3;
+            const uint64_t ad = smem_desc_sw128(sQ + (r * 2 + c) * fsm::kHalf + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sk + c * fsm::kHalf + kk * 32, 16, 1024);
+            mma_ss(tmem + r * 128, ad, bd, nb == 2 ? idS2 : idS1, k > 0 ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&bar_s[r]));
+        }
+        if (!ok) break;
+        for (int r = 0; r < n_tiles; ++r) {
+          if (!(ok = mbar_wait(smem_u32(&bar_p[r]), p & 1, abort_flag, a.err))) break;
+          tc_fence_after();
+          for (int j = 0; j < 4 * nb; ++j) {
+            const uint64_t bd = smem_desc_sw128(sv + j * 2048, fsm::kHalf, 1024);
+            mma_ts(tmem + 256 + r * 128, tmem + r * 128 + j * 8, bd, idPV, (p > 0 || j > 0) ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&bar_o[r]));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&bar_empty[st]));
+      }
+      mma_commit(smem_u32(&bar_fin));
+    }
+  } else if (warp >= 4 && (warp - 4) / 4 < n_tiles) {
+    // ------------------------------------------------------------ softmax, one row per thread
+    const int r = (warp - 4) / 4;
+    const int quarter = warp & 3;
+    const int row = 32 * quarter + lane;
+    const uint32_t lane_addr = uint32_t(32 * quarter) << 16;
+    const uint32_t tS = tmem + lane_addr + r * 128, tO = tmem + lane_addr + 256 + r * 128;
+    const int qpos = row & 63;
+    const float sc2 = a.scale * kLog2e;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int p = 0; p < n_pairs; ++p) {
+      ok = mbar_wait(smem_u32(&bar_s[r]), p & 1, abort_flag, a.err);
+      if (!__all_sync(0xffffffffu, ok)) {  // TMEM loads below are warp-collective
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int nb = min(2, nl - 2 * p);
+      const float lamA = lam_s[2 * p], lamB = nb > 1 ? lam_s[2 * p + 1] : 0.f;
+      const bool diag = (p == 0);
+      // pass 1: row max of the gated, masked logits
+      float mx = -INFINITY;
+      for (int ch = 0; ch < 2 * nb; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tS + ch * 32, v);
+        tmem_wait_ld();
+        const float lam = ch < 2 ? lamA : lamB;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int col = ch * 32 + e;
+          float z = fmaf(__uint_as_float(v[e]), sc2, lam);
+          if (diag && col < 64 && col > qpos) z = -INFINITY;
+          mx = fmaxf(mx, z);
+        }
+      }
+      // The stabiliser moves only when the row max grows by more than 2^8. The
+      // decision is per row, but the TMEM round trip that rescales O is a
+      // warp-collective instruction, so a warp runs it whenever any of its rows
+      // moved, with alpha = 1 for the rows that did not.
+      float alpha = 1.f;
+      const bool grow = mx > m_used + fsm::kRescale;
+      if (grow) {
+        alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - mx);
+        l *= alpha;
+        m_used = mx;
+      }
+      if (p > 0 && __any_sync(0xffffffffu, grow)) {
+        // O holds PV of earlier pairs, complete because S_r(p) completed after it
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t v[32];
+          tmem_ld32(tO + ch * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+          tmem_st32(tO + ch * 32, v);
+        }
+        tmem_wait_st();
+      }
+      // pass 2: probabilities, row sum, bf16 P over the consumed S columns
+      for (int ch2 = 0; ch2 < nb; ++ch2) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const int ch = ch2 * 2 + hlf;
+          uint32_t v[32];
+          tmem_ld32(tS + ch * 32, v);
+          tmem_wait_ld();
+          const float lam = ch < 2 ? lamA : lamB;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = ch * 32 + 2 * e;
+            float z0 = fmaf(__uint_as_float(v[2 * e]), sc2, lam);
+            float z1 = fmaf(__uint_as_float(v[2 * e + 1]), sc2, lam);
+            if (diag && col < 64 && col > qpos) z0 = -INFINITY;
+            if (diag && col + 1 < 64 && col + 1 > qpos) z1 = -INFINITY;
+            const float p0 = exp2f(z0 - m_used), p1 = exp2f(z1 - m_used);
+            l += p0 + p1;
+            pk[hlf * 16 + e] = pack_bf16x2(p0, p1);
+          }
+        }
+        tmem_st32(tS + ch2 * 32, pk);  // P columns [32 ch2, 32 ch2 + 32) lie in S columns already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_p[r]));
+    }
+    if (ok) ok = mbar_wait(smem_u32(&bar_o[r]), (n_pairs - 1) & 1, abort_flag, a.err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const int hh = row >> 6;
+      if (2 * r + hh < n_heads) {
+        const int hq = h * a.G + g_first + 2 * r + hh;
+        const size_t orow = (size_t(b) * a.Hq + hq) * a.N + size_t(t) * kBlock + qpos;
+        const float inv = 1.f / l;
+        uint4* og = reinterpret_cast<uint4*>(a.o + orow * 128);
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t v[32];
+          tmem_ld32(tO + ch * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
+            og[ch * 4 + q4] = w;
+          }
+        }
+        if (a.lse_o != nullptr) a.lse_o[orow] = (m_used + log2f(l)) * kLn2;
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {  // every MMA this CTA issued has completed
+      const long long t0 = clock64();
+      while (!mbar_try_wait(smem_u32(&bar_fin), 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] read in 64 x 64 boxes with the 128-byte swizzle.
+bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             const float* s, const int32_t* idx, const float* lse_s, uint16_t* o, float* lse_o,
+                             int* err, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  const uint64_t rq = uint64_t(sh.B) * sh.Hq * sh.N, rkv = uint64_t(sh.B) * sh.Hkv * sh.N;
+  if (!make_tmap_bf16_2d(&tq, q, rq, 128) || !make_tmap_bf16_2d(&tk, k, rkv, 128) ||
+      !make_tmap_bf16_2d(&tv, v, rkv, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e =
+      cudaFuncSetAttribute(fwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fsm::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  FwdSm100Args a;
+  a.idx = idx;
+  a.s = s;
+  a.lse_s = lse_s;
+  a.o = o;
+  a.lse_o = lse_o;
+  a.err = err;
+  a.B = sh.B;
+  a.Hq = sh.Hq;
+  a.Hkv = sh.Hkv;
+  a.G = sh.G;
+  a.N = sh.N;
+  a.NB = sh.NB;
+  a.K = sh.K;
+  a.gated = sh.gated;
+  a.n_tp = (sh.G + 3) / 4;
+  a.scale = sh.scale;
+  dim3 grid(sh.NB, sh.Hkv * a.n_tp, sh.B);
+  fwd_sm100_kernel<<<grid, fsm::kThreads, fsm::kSmemBytes, st>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace sas

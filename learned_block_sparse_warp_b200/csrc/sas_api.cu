@@ -12,6 +12,9 @@ cudaError_t launch_select(const Shape& sh, const float* s, const int32_t* cache_
 cudaError_t launch_fwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* s,
                            const int32_t* idx, const float* lse_s, uint16_t* o, float* lse_o, int* err,
                            cudaStream_t st);
+cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             const float* s, const int32_t* idx, const float* lse_s, uint16_t* o, float* lse_o,
+                             int* err, cudaStream_t st);
 struct BwdWs;
 size_t bwd_ws_layout(const Shape& sh, void* base, BwdWs* ws);
 cudaError_t launch_bwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -140,6 +143,10 @@ sas_status sas_fwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, co
   if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(idx) || !ok_ptr(o) || !ok_opt(lse_o))
     return SAS_ERR_INVALID_ARG;
   if (sh.gated && (!ok_ptr(s) || !ok_ptr(lse_s))) return SAS_ERR_INVALID_ARG;
+  // d = 128: TMA + tcgen05 kernel; d = 64: warp-level tensor-core kernel
+  if (sh.d == 128)
+    return from_cuda(sas::launch_fwd_sm100(sh, q, k, v, sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, o,
+                                           lse_o, device_error_word(), static_cast<cudaStream_t>(stream)));
   return from_cuda(sas::launch_fwd_mma(sh, q, k, v, sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, o, lse_o,
                                        device_error_word(), static_cast<cudaStream_t>(stream)));
 }

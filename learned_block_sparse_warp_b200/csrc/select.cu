@@ -67,17 +67,99 @@ __device__ void select_row(const float* __restrict__ row, int t, int K, int32_t*
   for (int k = written + lane; k < K; k += 32) idx[k] = -1;
 }
 
+// Register-resident variant for rows of at most 32·R scores: lane j holds
+// blocks j, j + 32, ... as order keys shifted up by one, so an empty slot (key
+// 0) never counts against a threshold. The search stops as soon as a
+// threshold isolates exactly n blocks.
+template <int R>
+__device__ void select_row_reg(const float* __restrict__ row, int t, int K, int32_t* __restrict__ idx,
+                               float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[R];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < R; ++j) {
+    const int m = lane + 32 * j;
+    const float f = (m < t) ? __ldg(row + m) : -INFINITY;
+    key[j] = (m < t) ? score_key(f) + 1u : 0u;
+    mx = fmaxf(mx, f);
+  }
+  if (lse != nullptr) {
+    mx = warp_max(mx);
+    float sum = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const int m = lane + 32 * j;
+        if (m < t) sum += expf(__ldg(row + m) - mx);
+      }
+    }
+    sum = warp_sum(sum);
+    if (lane == 0) *lse = (t == 0 || mx == -INFINITY) ? -INFINITY : mx + logf(sum);
+  }
+  if (idx == nullptr) return;
+  const int n = min(K, t);
+  uint32_t thr = 1u;  // every filled slot has key >= 1
+  bool exact = (n == t);
+  int need_eq = 0;
+  if (!exact) {
+    uint32_t acc = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = acc | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int j = 0; j < R; ++j) c += (key[j] >= cand) ? 1 : 0;
+      c = warp_isum(c);
+      if (c >= n) acc = cand;
+      if (c == n) {  // exactly n keys at or above cand: take them all
+        exact = true;
+        break;
+      }
+    }
+    thr = acc;
+    if (!exact) {
+      int gt = 0;
+#pragma unroll
+      for (int j = 0; j < R; ++j) gt += (key[j] > thr) ? 1 : 0;
+      need_eq = n - warp_isum(gt);
+    }
+  }
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int j = 0; j < R; ++j) {
+    if (32 * j >= t) break;
+    const uint32_t k = key[j];
+    const bool eq = !exact && k == thr;
+    const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_seen + __popc(eq_mask & ((1u << lane) - 1u));
+    const bool take = exact ? (k >= thr) : (k > thr || (eq && eq_rank < need_eq));
+    const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+    if (take) idx[written + __popc(take_mask & ((1u << lane) - 1u))] = lane + 32 * j;
+    written += __popc(take_mask);
+    eq_seen += __popc(eq_mask);
+  }
+  for (int k = written + lane; k < K; k += 32) idx[k] = -1;
+}
+
+template <int R>
+__device__ __forceinline__ void select_any(const float* row, int t, int K, int32_t* idx, float* lse) {
+  if (R > 0) select_row_reg<(R > 0 ? R : 1)>(row, t, K, idx, lse);
+  else select_row(row, t, K, idx, lse);
+}
+
 // Prefill: rows are (b, h, t) with t < NQB; row t reads s[b, h, t, 0..t).
+template <int R>
 __global__ void __launch_bounds__(256) select_prefill_kernel(const float* __restrict__ s, int rows, int NB, int K,
                                                              int32_t* __restrict__ idx, float* __restrict__ lse) {
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;
   const int t = r % NB;
-  select_row(s + size_t(r) * NB, t, K, idx ? idx + size_t(r) * K : nullptr, lse ? lse + r : nullptr);
+  select_any<R>(s + size_t(r) * NB, t, K, idx ? idx + size_t(r) * K : nullptr, lse ? lse + r : nullptr);
 }
 
 // Decode: rows are (b, h); the history of sequence b is blocks 0..c-1 with
 // c = (cache_len[b] - 1) / 64.
+template <int R>
 __global__ void __launch_bounds__(256) select_decode_kernel(const float* __restrict__ s,
                                                             const int32_t* __restrict__ cache_len, int B, int Hkv,
                                                             int NB, int K, int32_t* __restrict__ idx,
@@ -91,20 +173,30 @@ __global__ void __launch_bounds__(256) select_decode_kernel(const float* __restr
     if ((threadIdx.x & 31) == 0) raise_error(err, SAS_ERR_DEVICE_INDEX);
     c = 0;
   }
-  select_row(s + size_t(r) * NB, c, K, idx ? idx + size_t(r) * K : nullptr, lse ? lse + r : nullptr);
+  select_any<R>(s + size_t(r) * NB, c, K, idx ? idx + size_t(r) * K : nullptr, lse ? lse + r : nullptr);
+}
+
+template <int R>
+static void launch_select_r(const Shape& sh, const float* s, const int32_t* cache_len, int32_t* idx, float* lse,
+                            int* err, cudaStream_t st) {
+  const int warps = 8;
+  if (cache_len == nullptr) {
+    const int rows = sh.B * sh.Hkv * sh.NB;
+    select_prefill_kernel<R><<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(s, rows, sh.NB, sh.K, idx, lse);
+  } else {
+    const int rows = sh.B * sh.Hkv;
+    select_decode_kernel<R><<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(s, cache_len, sh.B, sh.Hkv, sh.NB,
+                                                                               sh.K, idx, lse, err);
+  }
 }
 
 cudaError_t launch_select(const Shape& sh, const float* s, const int32_t* cache_len, int32_t* idx, float* lse,
                           int* err, cudaStream_t st) {
-  const int warps = 8;
-  if (cache_len == nullptr) {
-    const int rows = sh.B * sh.Hkv * sh.NB;
-    select_prefill_kernel<<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(s, rows, sh.NB, sh.K, idx, lse);
-  } else {
-    const int rows = sh.B * sh.Hkv;
-    select_decode_kernel<<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(s, cache_len, sh.B, sh.Hkv, sh.NB, sh.K,
-                                                                            idx, lse, err);
-  }
+  // rows hold at most NB - 1 history scores
+  if (sh.NB <= 4 * 32) launch_select_r<4>(sh, s, cache_len, idx, lse, err, st);
+  else if (sh.NB <= 16 * 32) launch_select_r<16>(sh, s, cache_len, idx, lse, err, st);
+  else if (sh.NB <= 64 * 32) launch_select_r<64>(sh, s, cache_len, idx, lse, err, st);
+  else launch_select_r<0>(sh, s, cache_len, idx, lse, err, st);
   return cudaGetLastError();
 }
 
