@@ -439,23 +439,38 @@ __global__ void __launch_bounds__(256) bwd_ds_chain_kernel(const float* __restri
 // ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
+cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                   const uint16_t* dO, const float* s, const int32_t* idx, const float* lse_s,
+                                   const float* lse_o, const float* drow, const int* rev_off, const int* rev_list,
+                                   float* dl, uint16_t* dq, uint16_t* dk, uint16_t* dv, int* err, cudaStream_t st);
+
 template <int D>
 static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                 const uint16_t* o, const uint16_t* dO, const float* s, const int32_t* idx,
                                 const float* lse_s, const float* lse_o, uint16_t* dq, uint16_t* dk, uint16_t* dv,
-                                float* ds, void* ws_base, cudaStream_t st) {
+                                float* ds, void* ws_base, int* err, cudaStream_t st) {
   BwdWs ws;
   bwd_ws_layout(sh, ws_base, &ws);
   const size_t rows_q = size_t(sh.B) * sh.Hq * sh.N;
   const int nbh = sh.B * sh.Hkv;
   cudaError_t e;
-  if ((e = cudaMemsetAsync(ws.dq_acc, 0, rows_q * D * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(ws.dl, 0, size_t(nbh) * sh.NB * sh.K * sizeof(float), st)) != cudaSuccess) return e;
   bwd_prep_kernel<D><<<unsigned((rows_q + 7) / 8), 256, 0, st>>>(o, dO, rows_q, ws.drow);
   const int nw = nbh * sh.NB;
   revidx_count_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_cnt);
   revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
   revidx_fill_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_off, ws.rev_list);
+  if (D == 128) {  // tcgen05 passes: dK/dV/dl KV-major, then dQ query-major; no dQ accumulator
+    if ((e = launch_bwd_passes_sm100(sh, q, k, v, dO, s, idx, lse_s, lse_o, ws.drow, ws.rev_off, ws.rev_list, ws.dl,
+                                     dq, dk, dv, err, st)) != cudaSuccess)
+      return e;
+    if (ds != nullptr) {
+      const int rows = nbh * sh.NB;
+      bwd_ds_chain_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, lse_s, idx, ws.dl, rows, sh.NB, sh.K, sh.gated, ds);
+    }
+    return cudaGetLastError();
+  }
+  if ((e = cudaMemsetAsync(ws.dq_acc, 0, rows_q * D * sizeof(float), st)) != cudaSuccess) return e;
   const int smem = 6 * kBlock * D * 2 + 2 * kBlock * kBlock * 2;
   if ((e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
       cudaSuccess)
@@ -475,9 +490,9 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
 cudaError_t launch_bwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                            const uint16_t* o, const uint16_t* dO, const float* s, const int32_t* idx,
                            const float* lse_s, const float* lse_o, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* ds,
-                           void* ws, cudaStream_t st) {
-  if (sh.d == 128) return launch_bwd_d<128>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, st);
-  return launch_bwd_d<64>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, st);
+                           void* ws, int* err, cudaStream_t st) {
+  if (sh.d == 128) return launch_bwd_d<128>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, err, st);
+  return launch_bwd_d<64>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, err, st);
 }
 
 }  // namespace sas

@@ -20,7 +20,7 @@ size_t bwd_ws_layout(const Shape& sh, void* base, BwdWs* ws);
 cudaError_t launch_bwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                            const uint16_t* o, const uint16_t* dO, const float* s, const int32_t* idx,
                            const float* lse_s, const float* lse_o, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* ds,
-                           void* ws, cudaStream_t st);
+                           void* ws, int* err, cudaStream_t st);
 cudaError_t launch_decode(const Shape& sh, const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                           const int32_t* cl, const float* s, const int32_t* idx, const float* lse_s, int n_split,
                           float* o_part, float* lse_part, int* err, cudaStream_t st);
@@ -174,7 +174,8 @@ sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, co
   const size_t need = sas::bwd_ws_layout(sh, nullptr, nullptr);
   if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SAS_ERR_WORKSPACE;
   return from_cuda(sas::launch_bwd_mma(sh, q, k, v, o, dO, sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr,
-                                       lse_o, dq, dk, dv, ds, ws, static_cast<cudaStream_t>(stream)));
+                                       lse_o, dq, dk, dv, ds, ws, device_error_word(),
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_decode(const sas_params* p, const sas_bf16* q, const sas_bf16* kc, const sas_bf16* vc,
