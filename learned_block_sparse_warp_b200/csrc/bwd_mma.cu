@@ -37,6 +37,7 @@ struct BwdWs {
   int* rev_cnt;    // [B, Hkv, NB]
   int* rev_off;    // [B, Hkv, NB + 1]
   int* rev_list;   // [B, Hkv, NB * K]: (t << 8) | slot
+  float* rev_lam;  // [B, Hkv, NB * K]: log2-domain gate of each reverse-index entry
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -56,6 +57,8 @@ size_t bwd_ws_layout(const Shape& sh, void* base, BwdWs* ws) {
   off = align256(off + bhk * (sh.NB + 1) * sizeof(int));
   size_t o_list = off;
   off = align256(off + bhk * sh.NB * sh.K * sizeof(int));
+  size_t o_lam = off;
+  off = align256(off + bhk * sh.NB * sh.K * sizeof(float));
   if (ws != nullptr) {
     char* p = static_cast<char*>(base);
     ws->dq_acc = reinterpret_cast<float*>(p + o_dq);
@@ -64,6 +67,7 @@ size_t bwd_ws_layout(const Shape& sh, void* base, BwdWs* ws) {
     ws->rev_cnt = reinterpret_cast<int*>(p + o_cnt);
     ws->rev_off = reinterpret_cast<int*>(p + o_off);
     ws->rev_list = reinterpret_cast<int*>(p + o_list);
+    ws->rev_lam = reinterpret_cast<float*>(p + o_lam);
   }
   return off;
 }
@@ -139,7 +143,9 @@ __global__ void revidx_scan_kernel(const int* __restrict__ cnt, int NB, int* __r
 }
 
 __global__ void __launch_bounds__(256) revidx_fill_kernel(const int32_t* __restrict__ idx, int nbh, int NB, int K,
-                                                          const int* __restrict__ off, int* __restrict__ list) {
+                                                          const int* __restrict__ off, int* __restrict__ list,
+                                                          const float* __restrict__ s, const float* __restrict__ lse_s,
+                                                          int gated, float* __restrict__ lam) {
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (w >= nbh * NB) return;
   const int lane = threadIdx.x & 31;
@@ -151,7 +157,14 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const int32_t* __restr
     int slot = -1;
     if (t < NB) slot = find_slot(idx + (size_t(bh) * NB + t) * K, min(K, t), j);
     const unsigned mask = __ballot_sync(0xffffffffu, slot >= 0);
-    if (slot >= 0) out[pos + __popc(mask & ((1u << lane) - 1u))] = (t << 8) | slot;
+    if (slot >= 0) {
+      const int at = pos + __popc(mask & ((1u << lane) - 1u));
+      out[at] = (t << 8) | slot;
+      if (lam != nullptr) {  // the gate of block j for query block t, log2 domain
+        const size_t row = size_t(bh) * NB + t;
+        lam[size_t(bh) * NB * K + at] = gated ? (s[row * NB + j] - lse_s[row]) * kLog2e : 0.f;
+      }
+    }
     pos += __popc(mask);
   }
 }
@@ -442,7 +455,7 @@ __global__ void __launch_bounds__(256) bwd_ds_chain_kernel(const float* __restri
 cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                    const uint16_t* dO, const float* s, const int32_t* idx, const float* lse_s,
                                    const float* lse_o, const float* drow, const int* rev_off, const int* rev_list,
-                                   float* dl, uint16_t* dq, uint16_t* dk, uint16_t* dv, int* err, cudaStream_t st);
+                                   const float* rev_lam, float* dl, uint16_t* dq, uint16_t* dk, uint16_t* dv, int* err, cudaStream_t st);
 
 template <int D>
 static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -459,9 +472,11 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
   const int nw = nbh * sh.NB;
   revidx_count_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_cnt);
   revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
-  revidx_fill_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_off, ws.rev_list);
+  revidx_fill_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_off, ws.rev_list, s, lse_s,
+                                                    sh.gated, D == 128 ? ws.rev_lam : nullptr);
   if (D == 128) {  // tcgen05 passes: dK/dV/dl KV-major, then dQ query-major; no dQ accumulator
-    if ((e = launch_bwd_passes_sm100(sh, q, k, v, dO, s, idx, lse_s, lse_o, ws.drow, ws.rev_off, ws.rev_list, ws.dl,
+    if ((e = launch_bwd_passes_sm100(sh, q, k, v, dO, s, idx, lse_s, lse_o, ws.drow, ws.rev_off, ws.rev_list,
+                                     ws.rev_lam, ws.dl,
                                      dq, dk, dv, err, st)) != cudaSuccess)
       return e;
     if (ds != nullptr) {

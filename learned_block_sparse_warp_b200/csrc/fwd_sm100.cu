@@ -351,6 +351,33 @@ bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [heads, N, 128] read in boxes of 2 heads x 64 tokens x 64 d (128-byte swizzle), so one
+// load brings both heads of a head pair for one d-half: 128 rows of 128 B.
+bool make_tmap_bf16_3d_heads(CUtensorMap* m, const void* base, uint64_t heads, uint64_t N) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {128, N, heads};
+  const cuuint64_t strides[2] = {128 * 2, N * 128 * 2};
+  const cuuint32_t box[3] = {64, 64, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 [rows, N] read in boxes of 2 rows x 64 values (no swizzle).
+bool make_tmap_f32_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t N) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {N, rows};
+  const cuuint64_t strides[1] = {N * 4};
+  const cuuint32_t box[2] = {64, 2};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                              const float* s, const int32_t* idx, const float* lse_s, uint16_t* o, float* lse_o,
                              int* err, cudaStream_t st) {

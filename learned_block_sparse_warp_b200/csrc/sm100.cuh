@@ -72,6 +72,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// 3-D tile load: x = innermost coordinate (elements), then y, then z.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
 // 1-D bulk copy global -> shared, completion counted on `bar` (16-byte aligned, size % 16 == 0).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
@@ -110,6 +119,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
   d |= uint64_t(1) << 46;  // descriptor version for sm_100
   d |= uint64_t(2) << 61;  // SWIZZLE_128B
   return d;
+}
+
+// Adds a byte offset (a multiple of 16 that keeps the address field in range)
+// to a descriptor's start address.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) { return desc + uint64_t(bytes >> 4); }
+
+// 2^x on the special-function unit, flushing denormal results to zero.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Instruction descriptor of kind::f16 with bf16 A/B and an fp32 accumulator.
@@ -175,5 +195,9 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 // Row-major bf16 matrix [rows, cols] read in 64 x 64 boxes with the 128-byte swizzle (host).
 bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols);
+// bf16 [heads, N, 128] in boxes of 2 heads x 64 tokens x 64 d (host).
+bool make_tmap_bf16_3d_heads(CUtensorMap* m, const void* base, uint64_t heads, uint64_t N);
+// fp32 [rows, N] in boxes of 2 rows x 64 values (host).
+bool make_tmap_f32_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t N);
 
 }  // namespace sas
