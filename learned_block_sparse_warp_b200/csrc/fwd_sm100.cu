@@ -32,7 +32,7 @@
 namespace sas {
 
 namespace fsm {
-constexpr int kThreads = 384;
+constexpr int kThreads = 384;                    // 0 TMA, 1 and 3 MMA (one per tile), 4-11 softmax
 constexpr int kStages = 2;
 constexpr int kHalf = 128 * 128;                 // one d-half of a 128-row tile: 128 rows x 128 B
 constexpr int kQBytes = 4 * kHalf;               // 2 tiles x 2 d-halves
@@ -89,14 +89,14 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       mbar_init(smem_u32(&bar_q), 1);
       for (int s = 0; s < fsm::kStages; ++s) {
         mbar_init(smem_u32(&bar_full[s]), 1);
-        mbar_init(smem_u32(&bar_empty[s]), 1);
+        mbar_init(smem_u32(&bar_empty[s]), n_tiles);  // one commit per tile's MMA thread
       }
       for (int r = 0; r < 2; ++r) {
         mbar_init(smem_u32(&bar_s[r]), 1);
         mbar_init(smem_u32(&bar_p[r]), 128);
         mbar_init(smem_u32(&bar_o[r]), 1);
       }
-      mbar_init(smem_u32(&bar_fin), 1);
+      mbar_init(smem_u32(&bar_fin), n_tiles);
       fence_barrier_init();
     }
   }
@@ -145,44 +145,39 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if ((warp == 1 || warp == 3) && (warp >> 1) < n_tiles) {
+    // ------------------------------------------------------------ MMA issuers, one thread per tile
+    // (a single thread needs about 70 cycles per tcgen05.mma issue)
     if (lane == 0) {
+      const int r = warp >> 1;
       const uint32_t idS2 = idesc_bf16_f32(128, 128, 0, 0), idS1 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
+      const uint64_t dQ0 = smem_desc_sw128(sQ + r * 2 * fsm::kHalf, 16, 1024);
+      const uint64_t dK0 = smem_desc_sw128(sKV, 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(sKV + 2 * fsm::kHalf, fsm::kHalf, 1024);
+      const uint32_t tS = tmem + r * 128, tO = tmem + 256 + r * 128;
       bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, a.err);
       tc_fence_after();
       for (int p = 0; ok && p < n_pairs; ++p) {
         const int st = p % fsm::kStages, use = p / fsm::kStages;
         if (!(ok = mbar_wait(smem_u32(&bar_full[st]), use & 1, abort_flag, a.err))) break;
+        if (p > 0) {  // PV(p-1) reads P from the columns that S(p) overwrites
+          if (!(ok = mbar_wait(smem_u32(&bar_o[r]), (p - 1) & 1, abort_flag, a.err))) break;
+        }
         tc_fence_after();
         const int nb = min(2, nl - 2 * p);
-        const uint32_t sk = sKV + st * fsm::kStageBytes, sv = sk + 2 * fsm::kHalf;
-        for (int r = 0; r < n_tiles; ++r) {
-          if (p > 0) {  // PV_r(p-1) reads P_r from the columns that S_r(p) overwrites
-            if (!(ok = mbar_wait(smem_u32(&bar_o[r]), (p - 1) & 1, abort_flag, a.err))) break;
-            tc_fence_after();
-          }
+        const uint32_t so = st * fsm::kStageBytes;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int c = k >> 2, kk = k & 3;
-            const uint64_t ad = smem_desc_sw128(sQ + (r * 2 + c) * fsm::kHalf + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sk + c * fsm::kHalf + kk * 32, 16, 1024);
-            mma_ss(tmem + r * 128, ad, bd, nb == 2 ? idS2 : idS1, k > 0 ? 1u : 0u);
-          }
-          mma_commit(smem_u32(&bar_s[r]));
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t oc = (k >> 2) * fsm::kHalf + (k & 3) * 32;
+          mma_ss(tS, desc_advance(dQ0, oc), desc_advance(dK0, so + oc), nb == 2 ? idS2 : idS1, k > 0 ? 1u : 0u);
         }
-        if (!ok) break;
-        for (int r = 0; r < n_tiles; ++r) {
-          if (!(ok = mbar_wait(smem_u32(&bar_p[r]), p & 1, abort_flag, a.err))) break;
-          tc_fence_after();
-          for (int j = 0; j < 4 * nb; ++j) {
-            const uint64_t bd = smem_desc_sw128(sv + j * 2048, fsm::kHalf, 1024);
-            mma_ts(tmem + 256 + r * 128, tmem + r * 128 + j * 8, bd, idPV, (p > 0 || j > 0) ? 1u : 0u);
-          }
-          mma_commit(smem_u32(&bar_o[r]));
-        }
-        if (!ok) break;
+        mma_commit(smem_u32(&bar_s[r]));
+        if (!(ok = mbar_wait(smem_u32(&bar_p[r]), p & 1, abort_flag, a.err))) break;
+        tc_fence_after();
+        for (int jj = 0; jj < 4 * nb; ++jj)
+          mma_ts(tO, tS + jj * 8, desc_advance(dV0, so + jj * 2048), idPV, (p > 0 || jj > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&bar_o[r]));
         mma_commit(smem_u32(&bar_empty[st]));
       }
       mma_commit(smem_u32(&bar_fin));
@@ -207,22 +202,32 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       tc_fence_after();
       const int nb = min(2, nl - 2 * p);
       const float lamA = lam_s[2 * p], lamB = nb > 1 ? lam_s[2 * p + 1] : 0.f;
-      const bool diag = (p == 0);
-      // pass 1: row max of the gated, masked logits
-      float mx = -INFINITY;
+      const bool diag = (p == 0);  // block A of pair 0 is the causal current block
+      // pass 1: raw row max per 64-column block; the scale and gate are applied to the max
+      float rmA = -INFINITY, rmB = -INFINITY;
       for (int ch = 0; ch < 2 * nb; ++ch) {
         uint32_t v[32];
         tmem_ld32(tS + ch * 32, v);
         tmem_wait_ld();
-        const float lam = ch < 2 ? lamA : lamB;
+        float m0 = -INFINITY, m1 = -INFINITY;
+        if (diag && ch < 2) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = ch * 32 + e;
-          float z = fmaf(__uint_as_float(v[e]), sc2, lam);
-          if (diag && col < 64 && col > qpos) z = -INFINITY;
-          mx = fmaxf(mx, z);
+          for (int e = 0; e < 32; e += 2) {
+            if (ch * 32 + e <= qpos) m0 = fmaxf(m0, __uint_as_float(v[e]));
+            if (ch * 32 + e + 1 <= qpos) m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            m0 = fmaxf(m0, __uint_as_float(v[e]));
+            m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
+          }
         }
+        if (ch < 2) rmA = fmaxf(rmA, fmaxf(m0, m1));
+        else rmB = fmaxf(rmB, fmaxf(m0, m1));
       }
+      float mx = rmA == -INFINITY ? -INFINITY : fmaf(rmA, sc2, lamA);
+      if (nb > 1) mx = fmaxf(mx, fmaf(rmB, sc2, lamB));
       // The stabiliser moves only when the row max grows by more than 2^8. The
       // decision is per row, but the TMEM round trip that rescales O is a
       // warp-collective instruction, so a warp runs it whenever any of its rows
@@ -255,18 +260,22 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
           uint32_t v[32];
           tmem_ld32(tS + ch * 32, v);
           tmem_wait_ld();
-          const float lam = ch < 2 ? lamA : lamB;
+          const float off = (ch < 2 ? lamA : lamB) - m_used;  // p = 2^(S·sc2 + λ − m)
+          float pr[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pr[e] = fast_exp2(fmaf(__uint_as_float(v[e]), sc2, off));
+          if (diag && ch < 2) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pr[e] = (ch * 32 + e <= qpos) ? pr[e] : 0.f;
+          }
+          float s0 = 0.f, s1 = 0.f;
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int col = ch * 32 + 2 * e;
-            float z0 = fmaf(__uint_as_float(v[2 * e]), sc2, lam);
-            float z1 = fmaf(__uint_as_float(v[2 * e + 1]), sc2, lam);
-            if (diag && col < 64 && col > qpos) z0 = -INFINITY;
-            if (diag && col + 1 < 64 && col + 1 > qpos) z1 = -INFINITY;
-            const float p0 = exp2f(z0 - m_used), p1 = exp2f(z1 - m_used);
-            l += p0 + p1;
-            pk[hlf * 16 + e] = pack_bf16x2(p0, p1);
+            s0 += pr[2 * e];
+            s1 += pr[2 * e + 1];
+            pk[hlf * 16 + e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
           }
+          l += s0 + s1;
         }
         tmem_st32(tS + ch2 * 32, pk);  // P columns [32 ch2, 32 ch2 + 32) lie in S columns already read
       }
