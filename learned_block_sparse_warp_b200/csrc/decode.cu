@@ -12,33 +12,24 @@
 // the tasks' K, V and q rows through a multi-stage cp.async ring in shared
 // memory. Every CTA therefore keeps several 32 KB blocks in flight while it
 // computes on another, and there is no per-block launch or index-lookup
-// latency. The G query heads of a KV head share every K/V load (GQA grouping).
-// The task list (block index, token count, gate) is built in shared memory
-// before the ring starts, so no global load sits between two copies. The ring
-// uses only cp.async groups, with no spin-waits.
+// latency. The task list (block index, token count, gate) is built in shared
+// memory before the ring starts, so no global load sits between two copies.
+// The ring uses only cp.async groups, with no spin-waits.
+//
+// The arithmetic runs on mma.sync, so that the instruction count stays below
+// the memory time. The G <= 8 query heads of a KV head are padded to one
+// 16-row A fragment that serves every K/V load (GQA grouping). Each warp
+// scores 16 of the block's 64 tokens. Row maxima and sums are exchanged
+// through shared memory. P goes through a swizzled 16 x 64 bf16 tile, and
+// each warp then accumulates PV for a quarter of the head dimension.
 #include "common.cuh"
 
 namespace sas {
 
 namespace dec {
 constexpr int kThreads = 128;
-constexpr int kMaxTasks = 128;  // task slots per chunk of items
+constexpr int kMaxTasks = 64;   // task slots per chunk of items (keeps 2 CTAs per SM at d = 128)
 }  // namespace dec
-
-__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 r;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
-  return r;
-}
 
 struct DecodeArgs {
   const uint16_t* q;
@@ -57,33 +48,39 @@ struct DecodeArgs {
 
 template <int D, int G, int STAGES>
 __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs a) {
-  constexpr int CH = D / 8;            // 16-byte chunks per row
-  constexpr int ROWB = D * 2;          // bytes per K/V row
-  constexpr int TILEB = kBlock * ROWB;  // one 64-token tile
-  constexpr int QB = G * ROWB;          // the group's query rows
+  constexpr int CH = D / 8;             // 16-byte chunks per row
+  constexpr int ROWB = D * 2;           // bytes per K/V row
+  constexpr int TILEB = kBlock * ROWB;  // one 64-token tile, XOR-swizzled
+  constexpr int QB = 16 * ROWB;         // the group's query rows, padded to 16
   constexpr int STAGEB = 2 * TILEB + QB;
-  constexpr int LPR = CH;               // lanes per row: one 16-byte chunk each
-  constexpr int RPW = 32 / LPR;         // rows per warp per step
-  constexpr int RG = dec::kThreads / LPR;  // row groups in the PV product
+  constexpr int DW = D / 4;             // d columns per warp in PV
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int t_item[dec::kMaxTasks], t_m[dec::kMaxTasks], t_ntok[dec::kMaxTasks], t_flags[dec::kMaxTasks];
   __shared__ float t_lam[dec::kMaxTasks];
   __shared__ int n_tasks_s;
   __shared__ int cnt_s[dec::kThreads];
-  __shared__ float sc_s[G][kBlock];
-  __shared__ float m_s[G], l_s[G], a_s[G];
-  __shared__ float red_s[4][G][D];
+  __shared__ float red_max[4][8], red_sum[4][8];
+  __shared__ __align__(128) uint16_t p_s[16 * kBlock];  // P tile: 16 rows x 64 tokens, bf16, swizzled
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int NB = a.Lmax / kBlock;
   const int n_items = a.B * a.Hkv * a.n_split;
   const float sc2 = a.scale * kLog2e;
   const uint32_t ring = smem_u32(smem);
+  const uint32_t sP = smem_u32(p_s);
 
-  // this CTA's items: blockIdx.x + k * gridDim.x
+  // Stale shared memory must stay finite: masked products are 0 x value.
+  for (int i = tid; i < STAGES * STAGEB / 16; i += dec::kThreads)
+    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(ring + i * 16), "r"(0));
+  for (int i = tid; i < 16 * kBlock / 8; i += dec::kThreads)
+    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(sP + i * 16), "r"(0));
+  __syncthreads();
+
   const int my_items = (n_items > int(blockIdx.x)) ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+  const int g_row = lane >> 2;  // the head this thread's C-fragment row 0 belongs to
 
-  float acc[G][8];
+  float oacc[DW / 8][4];
+  float m_run = -INFINITY, l_run = 0.f;  // for head g_row (log2 domain), same in every warp
 
   for (int chunk0 = 0; chunk0 < my_items; chunk0 += a.items_per_chunk) {
     const int n_chunk = min(a.items_per_chunk, my_items - chunk0);
@@ -163,11 +160,14 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       const uint16_t* vb = a.vc + row0 * D;
       for (int i = tid; i < ntok * CH; i += dec::kThreads) {
         const int r = i / CH, ch = i % CH;
-        cp_async16(st + r * ROWB + ch * 16, kb + size_t(r) * D + ch * 8);
-        cp_async16(st + TILEB + r * ROWB + ch * 16, vb + size_t(r) * D + ch * 8);
+        cp_async16(st + swz<CH>(r, ch), kb + size_t(r) * D + ch * 8);
+        cp_async16(st + TILEB + swz<CH>(r, ch), vb + size_t(r) * D + ch * 8);
       }
-      const uint16_t* qb = a.q + size_t(bh) * G * D;
-      for (int i = tid; i < G * CH; i += dec::kThreads) cp_async16(st + 2 * TILEB + i * 16, qb + i * 8);
+      if (t_flags[task] & 1) {  // the item's first block brings its G query rows
+        const uint16_t* qb = a.q + size_t(bh) * G * D;
+        for (int i = tid; i < G * CH; i += dec::kThreads)
+          cp_async16(st + 2 * TILEB + swz<CH>(i / CH, i % CH), qb + (i / CH) * D + (i % CH) * 8);
+      }
     };
 
 #pragma unroll
@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       if (s < nt) issue(s);
       cp_async_commit();
     }
+    uint32_t qa[D / 16][4];  // A fragments of the padded query rows (rows >= G are zero)
     for (int task = 0; task < nt; ++task) {
       if (task + STAGES - 1 < nt) issue(task + STAGES - 1);
       cp_async_commit();
@@ -186,104 +187,94 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       const int flags = t_flags[task];
       if (flags & 1) {
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+        for (int j = 0; j < DW / 8; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+        m_run = -INFINITY;
+        l_run = 0.f;
+        // this stage holds the item's query rows; keep their A fragments in registers
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+        for (int kk = 0; kk < D / 16; ++kk)
+          ldsm_x4(st + 2 * TILEB + swz<CH>(lane & 15, 2 * kk + (lane >> 4)), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
       }
-      // scores: half-warps own rows, 16 lanes per row, one 16-byte chunk each
-      {
-        const int hh = lane / LPR, cl = lane % LPR;
-#pragma unroll 2
-        for (int i = 0; i < 16 / RPW; ++i) {
-          const int r = 16 * warp + RPW * i + hh;
-          float kf[8];
-          if (r < ntok) {
-            unpack8(lds128(st + r * ROWB + cl * 16), kf);
-          } else {
+      // S = q Kᵀ for this warp's 16 tokens (two n8 tiles); rows are heads
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) kf[e] = 0.f;
-          }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(st + swz<CH>(16 * warp + (lane & 7) + ((lane >> 4) << 3), 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
+        mma_bf16_16816(sacc[0], qa[kk], b0, b1);
+        mma_bf16_16816(sacc[1], qa[kk], b2, b3);
+      }
+      // gated logits (log2 domain) of head g_row; tokens past ntok are masked
+      float z[4];
+      float mx = -INFINITY;
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            float qf[8];
-            unpack8(lds128(st + 2 * TILEB + g * ROWB + cl * 16), qf);
-            float dot = 0.f;
+      for (int n = 0; n < 2; ++n)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
-#pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            if (cl == 0) sc_s[g][r] = (r < ntok) ? fmaf(dot, sc2, lam2) : -INFINITY;
-          }
+        for (int e = 0; e < 2; ++e) {
+          const int tok = 16 * warp + 8 * n + 2 * (lane & 3) + e;
+          const float v = tok < ntok ? fmaf(sacc[n][e], sc2, lam2) : -INFINITY;
+          z[2 * n + e] = v;
+          mx = fmaxf(mx, v);
         }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      if ((lane & 3) == 0 && g_row < 8) red_max[warp][g_row] = mx;
+      __syncthreads();
+      const float m_blk = fmaxf(fmaxf(red_max[0][g_row], red_max[1][g_row]), fmaxf(red_max[2][g_row], red_max[3][g_row]));
+      const float m_new = fmaxf(m_run, m_blk);
+      const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_new);
+      float ps = 0.f;
+      float pv[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        pv[x] = (z[x] == -INFINITY) ? 0.f : exp2f(z[x] - m_new);
+        ps += pv[x];
+      }
+      ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+      if ((lane & 3) == 0 && g_row < 8) red_sum[warp][g_row] = ps;
+      // P (bf16) of head g_row at tokens 16 warp + 8 n + 2 (lane & 3) + {0, 1}
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const int tok = 16 * warp + 8 * n + 2 * (lane & 3);
+        const uint32_t addr = sP + swz<8>(g_row, tok >> 3) + (tok & 7) * 2;
+        asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(addr), "r"(pack_bf16x2(pv[2 * n], pv[2 * n + 1])));
+      }
+#pragma unroll
+      for (int j = 0; j < DW / 8; ++j) {
+        oacc[j][0] *= alpha;
+        oacc[j][1] *= alpha;
       }
       __syncthreads();
-      // online softmax per head (one warp per head)
-      for (int g = warp; g < G; g += 4) {
-        const float z0 = sc_s[g][lane], z1 = sc_s[g][lane + 32];
-        const float m_old = (flags & 1) ? -INFINITY : m_s[g];
-        const float m_new = fmaxf(m_old, warp_max(fmaxf(z0, z1)));
-        const float p0 = (z0 == -INFINITY) ? 0.f : exp2f(z0 - m_new);
-        const float p1 = (z1 == -INFINITY) ? 0.f : exp2f(z1 - m_new);
-        const float bs = warp_sum(p0 + p1);
-        sc_s[g][lane] = p0;
-        sc_s[g][lane + 32] = p1;
-        if (lane == 0) {
-          const float alpha = (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
-          a_s[g] = alpha;
-          l_s[g] = ((flags & 1) ? 0.f : l_s[g]) * alpha + bs;
-          m_s[g] = m_new;
+      l_run = l_run * alpha + ((red_sum[0][g_row] + red_sum[1][g_row]) + (red_sum[2][g_row] + red_sum[3][g_row]));
+      m_run = m_new;
+      // O += P V over this warp's d columns [DW warp, DW warp + DW)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t pa[4];
+        ldsm_x4(sP + swz<8>(lane & 15, 2 * kk + (lane >> 4)), pa[0], pa[1], pa[2], pa[3]);
+#pragma unroll
+        for (int dp = 0; dp < DW / 16; ++dp) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(st + TILEB + swz<CH>(16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3), (DW / 8) * warp + 2 * dp + (lane >> 4)),
+                    b0, b1, b2, b3);
+          mma_bf16_16816(oacc[2 * dp], pa, b0, b1);
+          mma_bf16_16816(oacc[2 * dp + 1], pa, b2, b3);
         }
       }
-      __syncthreads();
-      // PV: 8 row groups of 16 lanes, one 16-byte chunk of d per lane
-      {
-        const int rg = tid / LPR, cl = tid % LPR;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float al = a_s[g];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[g][e] *= al;
-        }
-        for (int r = rg; r < ntok; r += RG) {
-          float vf[8];
-          unpack8(lds128(st + TILEB + r * ROWB + cl * 16), vf);
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float pw = sc_s[g][r];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pw, vf[e], acc[g][e]);
-          }
-        }
-      }
-      if (flags & 2) {  // last block of the item: reduce the row groups and write the partial
-        const int cl = tid % LPR;
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float v = acc[g][e];
-#pragma unroll
-            for (int o = LPR; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            acc[g][e] = v;
-          }
-        if (lane < LPR) {
-#pragma unroll
-          for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) red_s[warp][g][cl * 8 + e] = acc[g][e];
-        }
-        __syncthreads();
+      if (flags & 2) {  // the item's last block: write its normalised partial for the G heads
         const int it = t_item[task];
         const int split = it % a.n_split, bh = it / a.n_split;
-        for (int i = tid; i < G * D; i += dec::kThreads) {
-          const int g = i / D, e = i % D;
-          const float v = red_s[0][g][e] + red_s[1][g][e] + red_s[2][g][e] + red_s[3][g][e];
-          const float l = l_s[g];
-          a.o_part[((size_t(bh) * G + g) * a.n_split + split) * D + e] = (l > 0.f) ? v / l : 0.f;
-        }
-        if (tid < G) {
-          const float l = l_s[tid];
-          a.lse_part[(size_t(bh) * G + tid) * a.n_split + split] = (l > 0.f) ? (m_s[tid] + log2f(l)) * kLn2 : -INFINITY;
+        if (g_row < G) {
+          const size_t row = (size_t(bh) * G + g_row) * a.n_split + split;
+          const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+          for (int j = 0; j < DW / 8; ++j) {
+            const int col = DW * warp + 8 * j + 2 * (lane & 3);
+            *reinterpret_cast<float2*>(a.o_part + row * D + col) = make_float2(oacc[j][0] * inv, oacc[j][1] * inv);
+          }
+          if (warp == 0 && (lane & 3) == 0)
+            a.lse_part[row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         }
       }
       __syncthreads();
@@ -320,7 +311,7 @@ __global__ void decode_combine_kernel(const float* __restrict__ o_part, const fl
 template <int D, int G>
 static cudaError_t launch_decode_dg(const Shape& sh, const DecodeArgs& a, cudaStream_t st) {
   constexpr int STAGES = 3;
-  constexpr int smem = STAGES * (2 * kBlock * D * 2 + G * D * 2);
+  constexpr int smem = STAGES * (2 * kBlock * D * 2 + 16 * D * 2);
   auto kern = decode_split_kernel<D, G, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
