@@ -284,28 +284,65 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
   }
 }
 
+// One warp per (sequence, query head): the lanes read the split LSEs in
+// parallel, reduce them with shuffles, then stream the partials in float4s,
+// so no global load waits on another.
 template <int D>
-__global__ void decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                                      int n_split, uint16_t* __restrict__ o, float* __restrict__ lse_o) {
-  const size_t row = blockIdx.x;
-  const float* lp = lse_part + row * n_split;
+__global__ void __launch_bounds__(256) decode_combine_kernel(const float* __restrict__ o_part,
+                                                             const float* __restrict__ lse_part, int n_split,
+                                                             int rows, uint16_t* __restrict__ o,
+                                                             float* __restrict__ lse_o) {
+  constexpr int PER = D / 32;  // d values per lane: 4 or 2
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const float* lp = lse_part + size_t(row) * n_split;
   float mx = -INFINITY;
-  for (int j = 0; j < n_split; ++j) mx = fmaxf(mx, lp[j]);
+  for (int j = lane; j < n_split; j += 32) mx = fmaxf(mx, lp[j]);
+  mx = warp_max(mx);
   float den = 0.f;
   if (mx != -INFINITY)
-    for (int j = 0; j < n_split; ++j) den += exp2f((lp[j] - mx) * kLog2e);
-  const int e = threadIdx.x;
-  float acc = 0.f;
+    for (int j = lane; j < n_split; j += 32) den += exp2f((lp[j] - mx) * kLog2e);
+  den = warp_sum(den);
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   if (mx != -INFINITY) {
-    for (int j = 0; j < n_split; ++j) {
-      const float w = exp2f((lp[j] - mx) * kLog2e);
-      if (w > 0.f) acc = fmaf(w, o_part[(row * n_split + j) * D + e], acc);
+    const float* op = o_part + size_t(row) * n_split * D + lane * PER;
+    for (int j0 = 0; j0 < n_split; j0 += 32) {
+      const int jl = j0 + lane;
+      const float wl = (jl < n_split) ? exp2f((lp[jl] - mx) * kLog2e) : 0.f;  // weight of split jl
+      const int nj = min(32, n_split - j0);
+#pragma unroll 4
+      for (int u = 0; u < nj; ++u) {
+        const float w = __shfl_sync(0xffffffffu, wl, u);
+        if (w > 0.f) {
+          const float* src = op + size_t(j0 + u) * D;
+          if (PER == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src);
+            acc[0] = fmaf(w, x.x, acc[0]);
+            acc[1] = fmaf(w, x.y, acc[1]);
+            acc[PER > 2 ? 2 : 0] = fmaf(w, x.z, acc[PER > 2 ? 2 : 0]);
+            acc[PER > 3 ? 3 : 0] = fmaf(w, x.w, acc[PER > 3 ? 3 : 0]);
+          } else {
+            const float2 x = *reinterpret_cast<const float2*>(src);
+            acc[0] = fmaf(w, x.x, acc[0]);
+            acc[1] = fmaf(w, x.y, acc[1]);
+          }
+        }
+      }
     }
-    acc /= den;
+    const float inv = 1.f / den;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] *= inv;
   }
-  const __nv_bfloat16 r = __float2bfloat16_rn(acc);
-  o[row * D + e] = *reinterpret_cast<const uint16_t*>(&r);
-  if (lse_o != nullptr && e == 0) lse_o[row] = (mx == -INFINITY) ? -INFINITY : mx + logf(den);
+  uint16_t* dst = o + size_t(row) * D + lane * PER;
+  if (PER == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[PER > 2 ? 2 : 0], acc[PER > 3 ? 3 : 0]));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0], acc[1]);
+  }
+  if (lse_o != nullptr && lane == 0) lse_o[row] = (mx == -INFINITY) ? -INFINITY : mx + logf(den);
 }
 
 template <int D, int G>
@@ -374,9 +411,9 @@ cudaError_t launch_decode_combine(const Shape& sh, int n_split, const float* o_p
                                   uint16_t* o, float* lse_o, cudaStream_t st) {
   const int rows = sh.B * sh.Hq;
   if (sh.d == 128)
-    decode_combine_kernel<128><<<rows, 128, 0, st>>>(o_part, lse_part, n_split, o, lse_o);
+    decode_combine_kernel<128><<<(rows + 7) / 8, 256, 0, st>>>(o_part, lse_part, n_split, rows, o, lse_o);
   else
-    decode_combine_kernel<64><<<rows, 64, 0, st>>>(o_part, lse_part, n_split, o, lse_o);
+    decode_combine_kernel<64><<<(rows + 7) / 8, 256, 0, st>>>(o_part, lse_part, n_split, rows, o, lse_o);
   return cudaGetLastError();
 }
 

@@ -176,6 +176,129 @@ __global__ void __launch_bounds__(256) select_decode_kernel(const float* __restr
   select_any<R>(s + size_t(r) * NB, c, K, idx ? idx + size_t(r) * K : nullptr, lse ? lse + r : nullptr);
 }
 
+// One CTA of 256 threads per row, for few long rows (decode). Thread i holds
+// blocks i, i + 256, ... as shifted order keys in registers. Each threshold
+// candidate costs one __syncthreads_count per register slot, and the chosen
+// blocks are written in ascending order with block-wide ballot scans.
+constexpr int kRowThreads = 256;
+constexpr int kRowSlots = 8;  // rows of up to 2048 history blocks
+
+__device__ __forceinline__ int block_excl_scan(bool flag, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned m = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) warp_tot[warp] = __popc(m);
+  __syncthreads();
+  int before = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < kRowThreads / 32; ++w) {
+    const int c = warp_tot[w];
+    before += (w < warp) ? c : 0;
+    total += c;
+  }
+  __syncthreads();
+  return before + __popc(m & ((1u << lane) - 1u));
+}
+
+__global__ void __launch_bounds__(kRowThreads) select_decode_cta_kernel(const float* __restrict__ s,
+                                                                       const int32_t* __restrict__ cache_len,
+                                                                       int B, int Hkv, int NB, int K,
+                                                                       int32_t* __restrict__ idx,
+                                                                       float* __restrict__ lse, int* err) {
+  __shared__ int warp_tot[kRowThreads / 32];
+  __shared__ float red[kRowThreads / 32];
+  const int r = blockIdx.x;
+  const int b = r / Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int L = cache_len[b];
+  int t = (L - 1) / kBlock;
+  if (L < 1 || L > NB * kBlock) {
+    if (tid == 0) raise_error(err, SAS_ERR_DEVICE_INDEX);
+    t = 0;
+  }
+  const float* row = s + size_t(r) * NB;
+  uint32_t key[kRowSlots];
+  float f[kRowSlots];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int v = 0; v < kRowSlots; ++v) {
+    const int m = tid + kRowThreads * v;
+    f[v] = (m < t) ? __ldg(row + m) : -INFINITY;
+    key[v] = (m < t) ? score_key(f[v]) + 1u : 0u;
+    mx = fmaxf(mx, f[v]);
+  }
+  if (lse != nullptr) {
+    mx = warp_max(mx);
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    mx = red[0];
+#pragma unroll
+    for (int w = 1; w < kRowThreads / 32; ++w) mx = fmaxf(mx, red[w]);
+    __syncthreads();
+    float sum = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int v = 0; v < kRowSlots; ++v)
+        if (tid + kRowThreads * v < t) sum += expf(f[v] - mx);
+    }
+    sum = warp_sum(sum);
+    if (lane == 0) red[warp] = sum;
+    __syncthreads();
+    if (tid == 0) {
+      float tot = 0.f;
+      for (int w = 0; w < kRowThreads / 32; ++w) tot += red[w];
+      lse[r] = (t == 0 || mx == -INFINITY) ? -INFINITY : mx + logf(tot);
+    }
+  }
+  if (idx == nullptr) return;
+  int32_t* out = idx + size_t(r) * K;
+  const int n = min(K, t);
+  const int slots = (t + kRowThreads - 1) / kRowThreads;  // uniform
+  uint32_t thr = 1u;
+  bool exact = (n == t);
+  int need_eq = 0;
+  if (!exact) {
+    uint32_t acc = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = acc | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int v = 0; v < kRowSlots; ++v)
+        if (v < slots) c += __syncthreads_count(key[v] >= cand);  // slots is uniform over the block
+      if (c >= n) acc = cand;
+      if (c == n) {
+        exact = true;
+        break;
+      }
+    }
+    thr = acc;
+    if (!exact) {
+      int gt = 0;
+#pragma unroll
+      for (int v = 0; v < kRowSlots; ++v)
+        if (v < slots) gt += __syncthreads_count(key[v] > thr);
+      need_eq = n - gt;
+    }
+  }
+  // ascending order: slot-major, then thread
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int v = 0; v < kRowSlots; ++v) {
+    if (v >= slots) break;
+    const uint32_t k = key[v];
+    const bool eq = !exact && k == thr;
+    int eq_tot = 0;
+    const int eq_rank = eq_seen + block_excl_scan(eq, warp_tot, eq_tot);
+    const bool take = exact ? (k >= thr) : (k > thr || (eq && eq_rank < need_eq));
+    int take_tot = 0;
+    const int pos = written + block_excl_scan(take, warp_tot, take_tot);
+    if (take) out[pos] = tid + kRowThreads * v;
+    written += take_tot;
+    eq_seen += eq_tot;
+  }
+  for (int k = written + tid; k < K; k += kRowThreads) out[k] = -1;
+}
+
 template <int R>
 static void launch_select_r(const Shape& sh, const float* s, const int32_t* cache_len, int32_t* idx, float* lse,
                             int* err, cudaStream_t st) {
@@ -183,6 +306,9 @@ static void launch_select_r(const Shape& sh, const float* s, const int32_t* cach
   if (cache_len == nullptr) {
     const int rows = sh.B * sh.Hkv * sh.NB;
     select_prefill_kernel<R><<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(s, rows, sh.NB, sh.K, idx, lse);
+  } else if (sh.NB <= kRowThreads * kRowSlots) {  // decode: one CTA per (sequence, KV head)
+    select_decode_cta_kernel<<<sh.B * sh.Hkv, kRowThreads, 0, st>>>(s, cache_len, sh.B, sh.Hkv, sh.NB, sh.K, idx, lse,
+                                                                     err);
   } else {
     const int rows = sh.B * sh.Hkv;
     select_decode_kernel<R><<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(s, cache_len, sh.B, sh.Hkv, sh.NB,
