@@ -329,10 +329,12 @@ def run_gpu(args, rank, world, local_rank):
             "fwd_tflops": F / (fwd_ms * 1e-3) / 1e12,
             "bwd_tflops": achieved,
             "roofline": {"bound": "tensor",
-                         "kernel": "sas_bwd call (bwd_main_kernel + prep/reverse-index/epilogue)",
+                         "kernel": "sas_bwd call (KV pass + Q pass tcgen05 kernels, prep, reverse index, ds chain)",
                          "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16_sustained"], "peak_source": pk["source"] + " sustained bf16",
-                         "traffic": traffic_record("bwd_main", ["learned_block_sparse_warp_b200/csrc/bwd_mma.cu"])},
+                         "flops_per_launch": bwd_flops,
+                         "traffic": traffic_record("bwd_call", ["learned_block_sparse_warp_b200/csrc/bwd_mma.cu",
+                                                                "learned_block_sparse_warp_b200/csrc/bwd_sm100.cu"])},
             "e2e": e2e,
             "gpu_launches": args.steps * 9,
             "clocks": clk.summary(),
