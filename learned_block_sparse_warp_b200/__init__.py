@@ -24,6 +24,7 @@ __all__ = [
     "SAS_GATE_LOG_SOFTMAX", "SAS_GATE_NONE", "SasError", "Params", "lib",
     "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd", "sas_decode",
     "sas_decode_combine", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string", "sas_version",
+    "DecodeGraph",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
@@ -277,3 +278,28 @@ def decode_step(p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, str
     sas_decode(p, q, kc, vc, cache_len, s, out["idx"], out["lse_s"], n_split, out["o_part"], out["lse_part"],
                stream=stream)
     sas_decode_combine(p, n_split, out["o_part"], out["lse_part"], out["o"], out["lse_o"], stream=stream)
+
+
+class DecodeGraph:
+    """A decode step (select, split-K, merge) captured once as a CUDA graph.
+
+    The graph records the buffers' addresses, so a serving loop writes the
+    next step's query, scores and cache lengths into the same tensors and
+    calls ``replay()``. One replay is three kernel launches with no host work
+    between them. The three kernels are chained by programmatic dependent
+    launch, so each one's launch overlaps the tail of the one before.
+    """
+
+    def __init__(self, p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, stream=None):
+        self.args = (p, q, kc, vc, cache_len, s, n_split, out)
+        side = torch.cuda.Stream() if stream is None else stream
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):  # first call outside capture: kernel attributes get set here
+            decode_step(*self.args, stream=side)
+        torch.cuda.current_stream().wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=side, capture_error_mode="thread_local"):
+            decode_step(*self.args, stream=side)
+
+    def replay(self) -> None:
+        self.graph.replay()

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "sas.h"
 
 namespace sas {
@@ -80,7 +82,22 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint
 __device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr), "l"(gptr));
 }
+// Copies `src_bytes` (0 or 16) bytes and zero-fills the rest of the 16-byte chunk.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t smem_addr, const void* gptr, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_addr), "l"(gptr), "r"(src_bytes));
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start before its predecessor in the stream has finished;
+// griddep_wait() blocks until that predecessor has completed and its writes
+// are visible, so it must come before the first global access that could
+// depend on earlier work. Without that launch attribute it returns at once.
+// griddep_launch_dependents() lets the next such kernel begin its launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
@@ -135,6 +152,25 @@ __device__ __forceinline__ void build_block_list(const int32_t* __restrict__ idx
     lam_s[0] = 0.f;
     *nlist_s = 1 + cnt;
   }
+}
+
+// Launches `kern` with programmatic stream serialization, so that its launch
+// overlaps the tail of the preceding kernel. The kernel must call
+// griddep_wait() before its first global access.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace sas

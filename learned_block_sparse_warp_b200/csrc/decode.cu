@@ -22,6 +22,8 @@
 // scores 16 of the block's 64 tokens. Row maxima and sums are exchanged
 // through shared memory. P goes through a swizzled 16 x 64 bf16 tile, and
 // each warp then accumulates PV for a quarter of the head dimension.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace sas {
@@ -57,8 +59,7 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int t_item[dec::kMaxTasks], t_m[dec::kMaxTasks], t_ntok[dec::kMaxTasks], t_flags[dec::kMaxTasks];
   __shared__ float t_lam[dec::kMaxTasks];
-  __shared__ int n_tasks_s;
-  __shared__ int cnt_s[dec::kThreads];
+  __shared__ int wsum_s[dec::kThreads / 32];
   __shared__ float red_max[4][8], red_sum[4][8];
   __shared__ __align__(128) uint16_t p_s[16 * kBlock];  // P tile: 16 rows x 64 tokens, bf16, swizzled
 
@@ -69,12 +70,21 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
   const uint32_t ring = smem_u32(smem);
   const uint32_t sP = smem_u32(p_s);
 
-  // Stale shared memory must stay finite: masked products are 0 x value.
-  for (int i = tid; i < STAGES * STAGEB / 16; i += dec::kThreads)
-    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(ring + i * 16), "r"(0));
+  griddep_launch_dependents();  // the merge kernel may begin its launch; it waits for this grid's writes
+  // The padding rows G..15 of each stage's query tile and of the P tile are
+  // never loaded; they only feed output rows that are discarded, but are kept
+  // at zero so that every product stays finite. K/V rows past a block's token
+  // count are zero-filled by the copies themselves.
+  for (int i = tid; i < STAGES * (16 - G) * CH; i += dec::kThreads) {
+    const int stg = i / ((16 - G) * CH), rem = i % ((16 - G) * CH);
+    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(ring + stg * STAGEB + 2 * TILEB +
+                                                                  swz<CH>(G + rem / CH, rem % CH)),
+                 "r"(0));
+  }
   for (int i = tid; i < 16 * kBlock / 8; i += dec::kThreads)
     asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(sP + i * 16), "r"(0));
   __syncthreads();
+  griddep_wait();  // idx and lse_s come from the select kernel that precedes this one
 
   const int my_items = (n_items > int(blockIdx.x)) ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
   const int g_row = lane >> 2;  // the head this thread's C-fragment row 0 belongs to
@@ -109,22 +119,25 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
         }
       }
     }
-    cnt_s[tid] = cnt;
-    __syncthreads();
-    if (tid == 0) {  // exclusive scan of at most 128 counts
-      int run = 0;
-      for (int i = 0; i < dec::kThreads; ++i) {
-        const int v = cnt_s[i];
-        cnt_s[i] = run;
-        run += v;
-      }
-      n_tasks_s = run;
+    // exclusive scan of the per-item task counts: shuffles within a warp, then the warp totals
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
     }
+    if (lane == 31) wsum_s[warp] = incl;
     __syncthreads();
+    int base = incl - cnt, nt = 0;
+#pragma unroll
+    for (int w = 0; w < dec::kThreads / 32; ++w) {
+      const int v = wsum_s[w];
+      base += (w < warp) ? v : 0;
+      nt += v;
+    }
     if (tid < n_chunk) {
       const int bh = item / a.n_split;
       const float lse_bh = (a.gated && a.lse_s != nullptr) ? a.lse_s[bh] : 0.f;
-      const int base = cnt_s[tid];
       for (int j = 0; j < cnt; ++j) {
         const int pos = pos0 + j;
         int m = c, ntok = L - c * kBlock;
@@ -148,7 +161,6 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       }
     }
     __syncthreads();
-    const int nt = n_tasks_s;
 
     auto issue = [&](int task) {
       const uint32_t st = ring + (task % STAGES) * STAGEB;
@@ -158,10 +170,14 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       const size_t row0 = size_t(bh) * a.Lmax + size_t(t_m[task]) * kBlock;
       const uint16_t* kb = a.kc + row0 * D;
       const uint16_t* vb = a.vc + row0 * D;
-      for (int i = tid; i < ntok * CH; i += dec::kThreads) {
+      // rows past ntok are zero-filled (no bytes read), so masked tokens multiply finite zeros
+#pragma unroll 4
+      for (int i = tid; i < kBlock * CH; i += dec::kThreads) {
         const int r = i / CH, ch = i % CH;
-        cp_async16(st + swz<CH>(r, ch), kb + size_t(r) * D + ch * 8);
-        cp_async16(st + TILEB + swz<CH>(r, ch), vb + size_t(r) * D + ch * 8);
+        const int nb = r < ntok ? 16 : 0;
+        const size_t off = r < ntok ? size_t(r) * D + ch * 8 : 0;
+        cp_async16_zfill(st + swz<CH>(r, ch), kb + off, nb);
+        cp_async16_zfill(st + TILEB + swz<CH>(r, ch), vb + off, nb);
       }
       if (t_flags[task] & 1) {  // the item's first block brings its G query rows
         const uint16_t* qb = a.q + size_t(bh) * G * D;
@@ -284,61 +300,65 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
   }
 }
 
-// One warp per (sequence, query head): the lanes read the split LSEs in
-// parallel, reduce them with shuffles, then stream the partials in float4s,
-// so no global load waits on another.
+// One warp per (sequence, query head). The lanes read the split LSEs in
+// parallel and reduce them with shuffles. The partials are then streamed in
+// batches of 16 float4 (d = 128) or float2 (d = 64) loads per lane, all
+// issued before the first is used, so a batch costs one L2 round trip. The
+// weight is applied by a select, with no branch around the loads.
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const float* __restrict__ o_part,
                                                              const float* __restrict__ lse_part, int n_split,
                                                              int rows, uint16_t* __restrict__ o,
                                                              float* __restrict__ lse_o) {
   constexpr int PER = D / 32;  // d values per lane: 4 or 2
+  constexpr int BATCH = 16;
+  using VecT = typename std::conditional<PER == 4, float4, float2>::type;
+  griddep_wait();  // the partials come from the split kernel that precedes this one
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int lane = threadIdx.x & 31;
   const float* lp = lse_part + size_t(row) * n_split;
-  float mx = -INFINITY;
-  for (int j = lane; j < n_split; j += 32) mx = fmaxf(mx, lp[j]);
+  const float l0 = lane < n_split ? lp[lane] : -INFINITY;
+  float mx = l0;
+  for (int j = lane + 32; j < n_split; j += 32) mx = fmaxf(mx, lp[j]);
   mx = warp_max(mx);
-  float den = 0.f;
-  if (mx != -INFINITY)
-    for (int j = lane; j < n_split; j += 32) den += exp2f((lp[j] - mx) * kLog2e);
-  den = warp_sum(den);
+  const float mref = (mx == -INFINITY) ? 0.f : mx;  // all splits empty: every weight is 0
+  const float* op = o_part + size_t(row) * n_split * D + lane * PER;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  if (mx != -INFINITY) {
-    const float* op = o_part + size_t(row) * n_split * D + lane * PER;
-    for (int j0 = 0; j0 < n_split; j0 += 32) {
-      const int jl = j0 + lane;
-      const float wl = (jl < n_split) ? exp2f((lp[jl] - mx) * kLog2e) : 0.f;  // weight of split jl
-      const int nj = min(32, n_split - j0);
-#pragma unroll 4
-      for (int u = 0; u < nj; ++u) {
-        const float w = __shfl_sync(0xffffffffu, wl, u);
-        if (w > 0.f) {
-          const float* src = op + size_t(j0 + u) * D;
-          if (PER == 4) {
-            const float4 x = *reinterpret_cast<const float4*>(src);
-            acc[0] = fmaf(w, x.x, acc[0]);
-            acc[1] = fmaf(w, x.y, acc[1]);
-            acc[PER > 2 ? 2 : 0] = fmaf(w, x.z, acc[PER > 2 ? 2 : 0]);
-            acc[PER > 3 ? 3 : 0] = fmaf(w, x.w, acc[PER > 3 ? 3 : 0]);
-          } else {
-            const float2 x = *reinterpret_cast<const float2*>(src);
-            acc[0] = fmaf(w, x.x, acc[0]);
-            acc[1] = fmaf(w, x.y, acc[1]);
-          }
-        }
+  float den = 0.f;
+  for (int j0 = 0; j0 < n_split; j0 += 32) {
+    const int jl = j0 + lane;
+    const float l = j0 == 0 ? l0 : (jl < n_split ? lp[jl] : -INFINITY);
+    const float wl = exp2f((l - mref) * kLog2e);  // 0 for an empty split (lse = -inf)
+    den += wl;
+    const int nj = min(32, n_split - j0);
+    for (int u0 = 0; u0 < nj; u0 += BATCH) {
+      VecT x[BATCH];
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u) {
+        const int j = j0 + min(u0 + u, nj - 1);  // a valid split; surplus slots get weight 0
+        x[u] = *reinterpret_cast<const VecT*>(op + size_t(j) * D);
+      }
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u) {
+        const float w0 = __shfl_sync(0xffffffffu, wl, (u0 + u) & 31);
+        const float w = (u0 + u < nj && w0 > 0.f) ? w0 : 0.f;
+        const float* xv = reinterpret_cast<const float*>(&x[u]);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = w > 0.f ? fmaf(w, xv[e], acc[e]) : acc[e];
       }
     }
-    const float inv = 1.f / den;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] *= inv;
   }
+  den = warp_sum(den);
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] *= inv;
   uint16_t* dst = o + size_t(row) * D + lane * PER;
   if (PER == 4) {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[PER > 2 ? 2 : 0], acc[PER > 3 ? 3 : 0]));
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[PER > 2 ? 2 : 0], acc[PER > 3 ? 3 : 0]));
   } else {
     *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0], acc[1]);
   }
@@ -359,7 +379,8 @@ static cudaError_t launch_decode_dg(const Shape& sh, const DecodeArgs& a, cudaSt
     return e;
   const int n_items = a.B * a.Hkv * a.n_split;
   const int grid = max(1, min(n_items, sms * max(1, per_sm)));
-  kern<<<grid, dec::kThreads, smem, st>>>(a);
+  e = launch_pdl(kern, dim3(grid), dim3(dec::kThreads), smem, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -410,10 +431,11 @@ cudaError_t launch_decode(const Shape& sh, const uint16_t* q, const uint16_t* kc
 cudaError_t launch_decode_combine(const Shape& sh, int n_split, const float* o_part, const float* lse_part,
                                   uint16_t* o, float* lse_o, cudaStream_t st) {
   const int rows = sh.B * sh.Hq;
-  if (sh.d == 128)
-    decode_combine_kernel<128><<<(rows + 7) / 8, 256, 0, st>>>(o_part, lse_part, n_split, rows, o, lse_o);
-  else
-    decode_combine_kernel<64><<<(rows + 7) / 8, 256, 0, st>>>(o_part, lse_part, n_split, rows, o, lse_o);
+  const dim3 grid((rows + 7) / 8), block(256);
+  const cudaError_t e =
+      sh.d == 128 ? launch_pdl(decode_combine_kernel<128>, grid, block, 0, st, o_part, lse_part, n_split, rows, o, lse_o)
+                  : launch_pdl(decode_combine_kernel<64>, grid, block, 0, st, o_part, lse_part, n_split, rows, o, lse_o);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -164,6 +164,8 @@ __global__ void __launch_bounds__(256) select_decode_kernel(const float* __restr
                                                             const int32_t* __restrict__ cache_len, int B, int Hkv,
                                                             int NB, int K, int32_t* __restrict__ idx,
                                                             float* __restrict__ lse, int* err) {
+  griddep_wait();  // s and cache_len may come from the work just before this launch
+  griddep_launch_dependents();
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= B * Hkv) return;
   const int b = r / Hkv;
@@ -207,23 +209,31 @@ __global__ void __launch_bounds__(kRowThreads) select_decode_cta_kernel(const fl
                                                                        float* __restrict__ lse, int* err) {
   __shared__ int warp_tot[kRowThreads / 32];
   __shared__ float red[kRowThreads / 32];
+  griddep_wait();  // s and cache_len may come from the work just before this launch
+  griddep_launch_dependents();
   const int r = blockIdx.x;
   const int b = r / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* row = s + size_t(r) * NB;
+  // the whole row is read while cache_len is still in flight, then masked to the history
+  float f[kRowSlots];
+#pragma unroll
+  for (int v = 0; v < kRowSlots; ++v) {
+    const int m = tid + kRowThreads * v;
+    f[v] = (m < NB) ? __ldg(row + m) : -INFINITY;
+  }
   const int L = cache_len[b];
   int t = (L - 1) / kBlock;
   if (L < 1 || L > NB * kBlock) {
     if (tid == 0) raise_error(err, SAS_ERR_DEVICE_INDEX);
     t = 0;
   }
-  const float* row = s + size_t(r) * NB;
   uint32_t key[kRowSlots];
-  float f[kRowSlots];
   float mx = -INFINITY;
 #pragma unroll
   for (int v = 0; v < kRowSlots; ++v) {
     const int m = tid + kRowThreads * v;
-    f[v] = (m < t) ? __ldg(row + m) : -INFINITY;
+    if (m >= t) f[v] = -INFINITY;
     key[v] = (m < t) ? score_key(f[v]) + 1u : 0u;
     mx = fmaxf(mx, f[v]);
   }
@@ -307,12 +317,12 @@ static void launch_select_r(const Shape& sh, const float* s, const int32_t* cach
     const int rows = sh.B * sh.Hkv * sh.NB;
     select_prefill_kernel<R><<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(s, rows, sh.NB, sh.K, idx, lse);
   } else if (sh.NB <= kRowThreads * kRowSlots) {  // decode: one CTA per (sequence, KV head)
-    select_decode_cta_kernel<<<sh.B * sh.Hkv, kRowThreads, 0, st>>>(s, cache_len, sh.B, sh.Hkv, sh.NB, sh.K, idx, lse,
-                                                                     err);
+    launch_pdl(select_decode_cta_kernel, dim3(sh.B * sh.Hkv), dim3(kRowThreads), 0, st, s, cache_len, sh.B, sh.Hkv,
+               sh.NB, sh.K, idx, lse, err);
   } else {
     const int rows = sh.B * sh.Hkv;
-    select_decode_kernel<R><<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(s, cache_len, sh.B, sh.Hkv, sh.NB,
-                                                                               sh.K, idx, lse, err);
+    launch_pdl(select_decode_kernel<R>, dim3((rows + warps - 1) / warps), dim3(warps * 32), 0, st, s, cache_len, sh.B,
+               sh.Hkv, sh.NB, sh.K, idx, lse, err);
   }
 }
 

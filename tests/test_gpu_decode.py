@@ -53,22 +53,55 @@ def test_decode_parity(B, Hq, Hkv, d, Lmax, K, n_split, lens, gate):
     assert max_abs(host(out["lse_o"]), ref["lse"]) < TOL_L
 
 
-def test_combine_on_oracle_partials():
-    """The merge kernel alone, fed partials the oracle computed (including empty splits)."""
+@pytest.mark.parametrize("d,ns", [(128, 5), (128, 17), (64, 40), (128, 70), (128, 1)])
+def test_combine_on_oracle_partials(d, ns):
+    """The merge kernel alone, fed partials the oracle computed (including empty splits and rows)."""
     sas = _sas()
-    B, Hq, d, ns = 3, 4, 128, 5
-    g = np.random.default_rng(9)
+    B, Hq = 3, 4
+    g = np.random.default_rng(9 + ns)
     o_part = g.standard_normal((B, Hq, ns, d))
     lse_part = g.standard_normal((B, Hq, ns)) * 3
-    lse_part[0, 1, 2] = -np.inf
+    lse_part[0, 1, min(2, ns - 1)] = -np.inf
     lse_part[2, 3, :] = -np.inf
-    lse_part[2, 3, 4] = 0.5
+    lse_part[2, 3, ns - 1] = 0.5
+    lse_part[1, 2, :] = -np.inf  # a row with no tokens at all: o = 0, lse = -inf
     o_part[lse_part == -np.inf] = 0.0
-    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hq, head_dim=d, seq_len=1024, top_k=8)
+    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hq, head_dim=d, seq_len=1024, top_k=max(8, ns - 1))
     o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
     sas.sas_decode_combine(p, ns, f32_dev(o_part), f32_dev(lse_part), o, lse)
     torch.cuda.synchronize()
     ref_o, ref_lse = O.decode_combine(o_part, lse_part)
     assert max_abs(host(o), ref_o) < TOL_O
-    assert max_abs(host(lse), ref_lse) < 1e-5
+    got = host(lse)
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(np.isfinite(got), fin) and np.all(got[~fin] == -np.inf)
+    assert max_abs(got[fin], ref_lse[fin]) < 1e-5
+
+
+def test_decode_graph_replays_fresh_inputs():
+    """A captured decode step, replayed after its inputs change in place, matches the oracle."""
+    sas = _sas()
+    B, Hq, Hkv, d, Lmax, K, n_split = 4, 32, 8, 128, 2048, 8, 9
+    q, kc, vc, s = _case(B, Hq, Hkv, d, Lmax, seed=77)
+    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=Lmax, top_k=K,
+                   gate_mode=O.GATE_NONE)
+    out = sas.empty_decode_outputs(p, n_split)
+    qd, kd, vd, sd = bf16_dev(q), bf16_dev(kc), bf16_dev(vc), f32_dev(s)
+    cld = torch.tensor([2048, 700, 65, 1500], dtype=torch.int32, device="cuda")
+    graph = sas.DecodeGraph(p, qd, kd, vd, cld, sd, n_split, out)
+    for lens, seed in (([2048, 700, 65, 1500], None), ([1999, 1, 1024, 640], 5)):
+        if seed is not None:  # a new step: new query, new scores, new lengths, same buffers
+            q2, _, _, s2 = _case(B, Hq, Hkv, d, Lmax, seed=seed)
+            qd.copy_(bf16_dev(q2))
+            sd.copy_(f32_dev(s2))
+            cld.copy_(torch.tensor(lens, dtype=torch.int32))
+            q, s = q2, s2
+        graph.replay()
+        torch.cuda.synchronize()
+        assert sas.sas_get_device_error() == 0
+        ref = O.decode(q, kc, vc, np.array(lens, np.int32), s.astype(np.float64), K, gate_mode=O.GATE_NONE,
+                       n_split=n_split)
+        assert_idx_equal(out["idx"].cpu().numpy(), ref["idx"])
+        assert max_abs(host(out["o"]), ref["o"]) < TOL_O
+        assert max_abs(host(out["lse_o"]), ref["lse"]) < TOL_L
