@@ -203,28 +203,39 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       const int nb = min(2, nl - 2 * p);
       const float lamA = lam_s[2 * p], lamB = nb > 1 ? lam_s[2 * p + 1] : 0.f;
       const bool diag = (p == 0);  // block A of pair 0 is the causal current block
-      // pass 1: raw row max per 64-column block; the scale and gate are applied to the max
+      // The pair's S row (up to 128 columns) comes out of TMEM in four loads and
+      // one wait, and stays in registers. Raw row max per 64-column block; the
+      // scale and gate are applied to the max. The current block is causal.
+      uint32_t v[128];
+      tmem_ld32(tS, v);
+      tmem_ld32(tS + 32, v + 32);
+      if (nb > 1) {
+        tmem_ld32(tS + 64, v + 64);
+        tmem_ld32(tS + 96, v + 96);
+      }
+      tmem_wait_ld();
+      if (diag) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) v[e] = e <= qpos ? v[e] : __float_as_uint(-INFINITY);
+      }
       float rmA = -INFINITY, rmB = -INFINITY;
-      for (int ch = 0; ch < 2 * nb; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tS + ch * 32, v);
-        tmem_wait_ld();
+      {
         float m0 = -INFINITY, m1 = -INFINITY;
-        if (diag && ch < 2) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            if (ch * 32 + e <= qpos) m0 = fmaxf(m0, __uint_as_float(v[e]));
-            if (ch * 32 + e + 1 <= qpos) m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            m0 = fmaxf(m0, __uint_as_float(v[e]));
-            m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
-          }
+        for (int e = 0; e < 64; e += 2) {
+          m0 = fmaxf(m0, __uint_as_float(v[e]));
+          m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
         }
-        if (ch < 2) rmA = fmaxf(rmA, fmaxf(m0, m1));
-        else rmB = fmaxf(rmB, fmaxf(m0, m1));
+        rmA = fmaxf(m0, m1);
+      }
+      if (nb > 1) {
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int e = 64; e < 128; e += 2) {
+          m0 = fmaxf(m0, __uint_as_float(v[e]));
+          m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
+        }
+        rmB = fmaxf(m0, m1);
       }
       float mx = rmA == -INFINITY ? -INFINITY : fmaf(rmA, sc2, lamA);
       if (nb > 1) mx = fmaxf(mx, fmaf(rmB, sc2, lamB));
@@ -239,45 +250,32 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         l *= alpha;
         m_used = mx;
       }
+      // probabilities, row sum, bf16 P over the S columns (all read above)
+      for (int ch2 = 0; ch2 < nb; ++ch2) {
+        const float off = (ch2 == 0 ? lamA : lamB) - m_used;  // p = 2^(S·sc2 + λ − m)
+        uint32_t pk[32];
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(v[64 * ch2 + 2 * e]), sc2, off));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(v[64 * ch2 + 2 * e + 1]), sc2, off));
+          s0 += p0;
+          s1 += p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        l += s0 + s1;
+        tmem_st32(tS + ch2 * 32, pk);  // P columns [32 ch2, 32 ch2 + 32)
+      }
       if (p > 0 && __any_sync(0xffffffffu, grow)) {
         // O holds PV of earlier pairs, complete because S_r(p) completed after it
         for (int ch = 0; ch < 4; ++ch) {
-          uint32_t v[32];
-          tmem_ld32(tO + ch * 32, v);
+          uint32_t w[32];
+          tmem_ld32(tO + ch * 32, w);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-          tmem_st32(tO + ch * 32, v);
+          for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * alpha);
+          tmem_st32(tO + ch * 32, w);
         }
-        tmem_wait_st();
-      }
-      // pass 2: probabilities, row sum, bf16 P over the consumed S columns
-      for (int ch2 = 0; ch2 < nb; ++ch2) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          const int ch = ch2 * 2 + hlf;
-          uint32_t v[32];
-          tmem_ld32(tS + ch * 32, v);
-          tmem_wait_ld();
-          const float off = (ch < 2 ? lamA : lamB) - m_used;  // p = 2^(S·sc2 + λ − m)
-          float pr[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pr[e] = fast_exp2(fmaf(__uint_as_float(v[e]), sc2, off));
-          if (diag && ch < 2) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) pr[e] = (ch * 32 + e <= qpos) ? pr[e] : 0.f;
-          }
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            s0 += pr[2 * e];
-            s1 += pr[2 * e + 1];
-            pk[hlf * 16 + e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
-          }
-          l += s0 + s1;
-        }
-        tmem_st32(tS + ch2 * 32, pk);  // P columns [32 ch2, 32 ch2 + 32) lie in S columns already read
       }
       tmem_wait_st();
       tc_fence_before();
