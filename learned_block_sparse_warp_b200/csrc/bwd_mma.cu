@@ -26,6 +26,8 @@
 //                    atomics.
 //   bwd_dq_convert   fp32 dQ -> bf16
 //   bwd_ds_chain     ds from dl through the softmax over s
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace sas {
@@ -73,22 +75,45 @@ size_t bwd_ws_layout(const Shape& sh, void* base, BwdWs* ws) {
 }
 
 // ---------------------------------------------------------------------------
-// D_i = dO_i · o_i (one warp per row)
+// D_i = dO_i · o_i. HBM-bound: each thread reads 16-byte chunks of o and dO,
+// a row is 256 (d = 128) or 128 bytes, so 16 or 8 lanes share a row and reduce
+// with shuffles. Each thread keeps four rows' loads in flight.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dO,
                                                        size_t rows, float* __restrict__ drow) {
-  const size_t r = size_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (r >= rows) return;
+  constexpr int CPR = D / 8;     // 16-byte chunks per row
+  constexpr int RPW = 32 / CPR;  // rows per warp and unroll step
+  constexpr int U = 4;
   const int lane = threadIdx.x & 31;
-  constexpr int PER = D / 32;  // 2 or 4 bf16 per lane
-  float acc = 0.f;
-  const uint16_t* po = o + r * D + lane * PER;
-  const uint16_t* pd = dO + r * D + lane * PER;
+  const int c = lane % CPR, sub = lane / CPR;
+  const size_t warp_g = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const size_t n_warps = (size_t(gridDim.x) * blockDim.x) >> 5;
+  const uint4* o4 = reinterpret_cast<const uint4*>(o);
+  const uint4* d4 = reinterpret_cast<const uint4*>(dO);
+  for (size_t r0 = warp_g * RPW * U; r0 < rows; r0 += n_warps * RPW * U) {
+    uint4 x[U], y[U];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) acc = fmaf(bf16_to_f32(po[e]), bf16_to_f32(pd[e]), acc);
-  acc = warp_sum(acc);
-  if (lane == 0) drow[r] = acc;
+    for (int u = 0; u < U; ++u) {
+      const size_t r = r0 + u * RPW + sub;
+      x[u] = r < rows ? __ldg(o4 + r * CPR + c) : make_uint4(0, 0, 0, 0);
+      y[u] = r < rows ? __ldg(d4 + r * CPR + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t xa[4] = {x[u].x, x[u].y, x[u].z, x[u].w}, ya[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc = fmaf(__uint_as_float(xa[k] << 16), __uint_as_float(ya[k] << 16), acc);
+        acc = fmaf(__uint_as_float(xa[k] & 0xffff0000u), __uint_as_float(ya[k] & 0xffff0000u), acc);
+      }
+#pragma unroll
+      for (int off = CPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const size_t r = r0 + u * RPW + sub;
+      if (c == 0 && r < rows) drow[r] = acc;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -468,7 +493,13 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
   const int nbh = sh.B * sh.Hkv;
   cudaError_t e;
   if ((e = cudaMemsetAsync(ws.dl, 0, size_t(nbh) * sh.NB * sh.K * sizeof(float), st)) != cudaSuccess) return e;
-  bwd_prep_kernel<D><<<unsigned((rows_q + 7) / 8), 256, 0, st>>>(o, dO, rows_q, ws.drow);
+  {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t rows_per_cta = size_t(8) * (32 / (D / 8)) * 4;  // warps x rows per warp step x unroll
+    const unsigned grid = unsigned(std::min<size_t>((rows_q + rows_per_cta - 1) / rows_per_cta, size_t(sms) * 8));
+    bwd_prep_kernel<D><<<std::max(1u, grid), 256, 0, st>>>(o, dO, rows_q, ws.drow);
+  }
   const int nw = nbh * sh.NB;
   revidx_count_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_cnt);
   revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
