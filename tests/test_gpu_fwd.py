@@ -47,6 +47,12 @@ CASES = [
     ("one_block", 2, 2, 2, 128, 64, 4),      # t = 0 only
     ("k1", 1, 4, 4, 64, 640, 1),
     ("batch3_d64_gqa2", 3, 4, 2, 64, 256, 2),
+    # tcgen05 paths (d = 128): one head per head pair, batch 2, eight heads with every block
+    # selected, and an odd group with K = 1
+    ("g1_d128", 1, 3, 3, 128, 512, 4),
+    ("g2_d128_b2", 2, 4, 2, 128, 512, 5),
+    ("g8_d128_dense", 1, 8, 1, 128, 512, 16),
+    ("g3_d128_k1", 1, 6, 2, 128, 640, 1),
 ]
 
 
