@@ -60,8 +60,11 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
   __shared__ int list_s[kMaxTopK + 1];
   __shared__ float lam_s[kMaxTopK + 1];
   __shared__ int nlist_s;
+  // bar_turn[r]: tile r's softmax may run its exponentials. The two tiles take
+  // turns, so one tile's exponentials overlap the other tile's MMAs instead of
+  // both contending for the SM's exponential units at once.
   __shared__ __align__(8) uint64_t bar_q, bar_full[fsm::kStages], bar_empty[fsm::kStages], bar_s[2], bar_p[2],
-      bar_o[2], bar_fin;
+      bar_o[2], bar_fin, bar_turn[2];
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
 
@@ -97,6 +100,8 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         mbar_init(smem_u32(&bar_o[r]), 1);
       }
       mbar_init(smem_u32(&bar_fin), n_tiles);
+      mbar_init(smem_u32(&bar_turn[0]), 4);  // one arrival per softmax warp of the other tile
+      mbar_init(smem_u32(&bar_turn[1]), 4);
       fence_barrier_init();
     }
   }
@@ -250,6 +255,16 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         l *= alpha;
         m_used = mx;
       }
+      // Turn order: tile 0 pair 0, tile 1 pair 0, tile 0 pair 1, ... Tile 0 waits for
+      // tile 1's turn of pair p - 1, tile 1 for tile 0's turn of pair p. Neither
+      // barrier can run a phase ahead: its next phase needs the waiter's own turn.
+      if (n_tiles == 2 && (r == 1 || p > 0)) {
+        const bool got = mbar_wait(smem_u32(&bar_turn[r]), (r == 0 ? p - 1 : p) & 1, abort_flag, a.err);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+      }
       // probabilities, row sum, bf16 P over the S columns (all read above)
       for (int ch2 = 0; ch2 < nb; ++ch2) {
         const float off = (ch2 == 0 ? lamA : lamB) - m_used;  // p = 2^(S·sc2 + λ − m)
@@ -280,6 +295,10 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&bar_p[r]));
+      if (n_tiles == 2) {  // pass the turn to the other tile
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_turn[r ^ 1]));
+      }
     }
     if (ok) ok = mbar_wait(smem_u32(&bar_o[r]), (n_pairs - 1) & 1, abort_flag, a.err);
     ok = __all_sync(0xffffffffu, ok);
