@@ -194,6 +194,52 @@ def oracle_baseline(w, budget_s=15.0):
 
 
 # ---------------------------------------------------------------------------
+# ranks: one process per GPU, replicas of the workload, no collective on the data path
+# ---------------------------------------------------------------------------
+def rank_env(env=None):
+    """(rank, world, local_rank) from the torch.distributed.run environment (one rank without it)."""
+    env = os.environ if env is None else env
+    return int(env.get("RANK", 0)), int(env.get("WORLD_SIZE", 1)), int(env.get("LOCAL_RANK", 0))
+
+
+def relaunch_command(gpus: int, argv, port: int):
+    """The torch.distributed.run command that runs this script with one rank per GPU."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
+def init_ranks(world: int, backend: str, device=None, timeout_s: float = 120.0):
+    """The process group for the barrier and the max-over-ranks timing, or None for one rank."""
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    kw = {"device_id": device} if backend == "nccl" and device is not None else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return dist
+
+
+def barrier(dist) -> None:
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, x: float, device="cpu") -> float:
+    """The slowest rank's value: every rank takes the same all-reduce, in the same order."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput of weak-scaled replicas: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank / max_seconds
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 def run_gpu(args, rank, world, local_rank):
@@ -204,22 +250,7 @@ def run_gpu(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    dist = init_ranks(world, "nccl", dev)
 
     stream = torch.cuda.Stream(device=dev)
     pk = peaks()
@@ -255,7 +286,7 @@ def run_gpu(args, rank, world, local_rank):
             torch.cuda.synchronize()
             if sas.sas_get_device_error(stream) != 0:
                 raise RuntimeError("device error during warm-up")
-            barrier()
+            barrier(dist)
             torch.cuda.synchronize()
             clk.mark("t_begin")
             t_start = torch.cuda.Event(enable_timing=True)
@@ -267,8 +298,8 @@ def run_gpu(args, rank, world, local_rank):
             torch.cuda.synchronize()
             clk.mark("t_end")
             time.sleep(0.25)
-        barrier()
-        total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+        barrier(dist)
+        total_ms = max_over_ranks(dist, t_start.elapsed_time(t_end), dev)
         sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
         fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
         bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -299,7 +330,7 @@ def run_gpu(args, rank, world, local_rank):
             e2e_step()
             torch.cuda.synchronize()
             n_e2e = max(1, min(args.steps, 3))
-            barrier()
+            barrier(dist)
             torch.cuda.synchronize()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
@@ -308,15 +339,15 @@ def run_gpu(args, rank, world, local_rank):
                 e2e_step()
             b.record(stream)
             torch.cuda.synchronize()
-            e2e_ms = max_over_ranks(a.elapsed_time(b)) / n_e2e
-            e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            e2e_ms = max_over_ranks(dist, a.elapsed_time(b), dev) / n_e2e
+            e2e = {"value": job_rate(step_flops, world, e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e}
             del h_in, d_in, h_out
 
         bwd_flops = 2.5 * F
         achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
         line.update({
-            "metric": METRIC, "value": world * step_flops * args.steps / (total_ms * 1e-3) / 1e12,
+            "metric": METRIC, "value": job_rate(step_flops * args.steps, world, total_ms * 1e-3) / 1e12,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -398,12 +429,12 @@ def run_gpu(args, rank, world, local_rank):
                     timings[key].append(fn())
         torch.cuda.synchronize()
         med = {key: statistics.median(e[0].elapsed_time(e[1]) for e in evs) for key, evs in timings.items()}
-        step_ms = max_over_ranks(med["step"])
+        step_ms = max_over_ranks(dist, med["step"], dev)
         split_ms = med["split"]
         kv = decode_kv_bytes(wd, xd["cache_len"].cpu().numpy())
         gbs = kv / (split_ms * 1e-3) / 1e9
         line["decode"] = {
-            "workload": DECODE, "tok_per_s": world * wd.batch / (step_ms * 1e-3), "ms_per_step": step_ms,
+            "workload": DECODE, "tok_per_s": job_rate(wd.batch, world, step_ms * 1e-3), "ms_per_step": step_ms,
             "launch": "CUDA graph of the three kernels, chained by programmatic dependent launch",
             "eager_ms_per_step": med["eager"], "select_ms": med["select"], "split_ms": split_ms,
             "combine_ms": med["combine"], "n_split": n_split,
@@ -468,11 +499,13 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    rank = int(os.environ.get("RANK", 0))
-    world = int(os.environ.get("WORLD_SIZE", 1))
-    local_rank = int(os.environ.get("LOCAL_RANK", 0))
-    if world != args.gpus:
-        world = args.gpus if "WORLD_SIZE" not in os.environ else world
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:  # one rank per GPU under torch.distributed.run
+        import socket
+        with socket.socket() as sock:
+            sock.bind(("127.0.0.1", 0))
+            port = sock.getsockname()[1]
+        sys.exit(subprocess.call(relaunch_command(args.gpus, sys.argv[1:], port)))
+    rank, world, local_rank = rank_env()
     if args.impl == "reference":
         line = run_reference(args, rank, world)
     else:
