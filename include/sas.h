@@ -196,6 +196,25 @@ SAS_API sas_status sas_decode(const sas_params* p, const sas_bf16* q, const sas_
                       const int32_t* cache_len, const float* s, const int32_t* idx, const float* lse_s, int n_split,
                       float* o_part, float* lse_part, void* stream);
 
+/* The same split-K decode over a paged KV cache (serving layout). A page holds
+ * one 64-token block of every KV head, and a block table maps each sequence's
+ * logical blocks to pages, so sequences grow without moving their history.
+ *   k_pages, v_pages  bf16 [n_pages, Hkv, 64, d]
+ *   n_pages           >= 1
+ *   block_table       int32 [B, NKB] with NKB = seq_len / 64: the page of
+ *                     logical block m of sequence b. Only the entries of the
+ *                     blocks the step reads (the current block and the
+ *                     selected history blocks) are read. An entry outside
+ *                     [0, n_pages) raises SAS_ERR_DEVICE_INDEX, and page 0 is
+ *                     read in its place.
+ *   seq_len           bounds cache_len, as Lmax does for sas_decode.
+ * Tokens of the current block's page past cache_len are never read. Every other
+ * argument and output is as in sas_decode. */
+SAS_API sas_status sas_decode_paged(const sas_params* p, const sas_bf16* q, const sas_bf16* k_pages,
+                                    const sas_bf16* v_pages, int n_pages, const int32_t* block_table,
+                                    const int32_t* cache_len, const float* s, const int32_t* idx, const float* lse_s,
+                                    int n_split, float* o_part, float* lse_part, void* stream);
+
 /* Merge of the split partials:
  *   LSE = log Σ_j exp lse_part[j],   o = Σ_j exp(lse_part[j] − LSE) · o_part[j].
  *   o      bf16 [B, Hq, d]. Output.

@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "SAS_GATE_LOG_SOFTMAX", "SAS_GATE_NONE", "SasError", "Params", "lib",
     "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd", "sas_decode",
-    "sas_decode_combine", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string", "sas_version",
+    "sas_decode_combine", "sas_decode_paged", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string",
+    "sas_version",
     "DecodeGraph",
 ]
 
@@ -63,6 +64,7 @@ def _load() -> ctypes.CDLL:
         "sas_bwd_workspace_size": [P, ctypes.POINTER(sz)],
         "sas_bwd": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "sas_decode": [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp],
+        "sas_decode_paged": [P, vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp],
         "sas_decode_combine": [P, ctypes.c_int, vp, vp, vp, vp, vp],
         "sas_get_device_error": [vp, ctypes.POINTER(ctypes.c_int)],
         "sas_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp],
@@ -205,6 +207,21 @@ def sas_decode(p: Params, q, kc, vc, cache_len, s, idx, lse_s, n_split: int, o_p
         _ptr(lse_part, f32, (B, Hq, n_split), "lse_part"), _stream(stream)))
 
 
+def sas_decode_paged(p: Params, q, k_pages, v_pages, block_table, cache_len, s, idx, lse_s, n_split: int, o_part,
+                     lse_part, stream=None) -> None:
+    """sas_decode over a paged cache: k_pages/v_pages [n_pages, Hkv, 64, d], block_table int32 [B, NKB]."""
+    B, Hq, Hkv, d = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim
+    n_pages = int(k_pages.shape[0]) if k_pages is not None else 0
+    sh = _shapes(p, True)
+    _check("sas_decode_paged", lib.sas_decode_paged(
+        ctypes.byref(p.c()), _ptr(q, bf16, (B, Hq, d), "q"), _ptr(k_pages, bf16, (n_pages, Hkv, p.block, d), "k_pages"),
+        _ptr(v_pages, bf16, (n_pages, Hkv, p.block, d), "v_pages"), n_pages,
+        _ptr(block_table, i32, (B, p.n_blocks), "block_table"), _ptr(cache_len, i32, (B,), "cache_len"),
+        _ptr(s, f32, sh["s"], "s"), _ptr(idx, i32, sh["idx"], "idx"), _ptr(lse_s, f32, sh["lse_s"], "lse_s"),
+        int(n_split), _ptr(o_part, f32, (B, Hq, n_split, d), "o_part"),
+        _ptr(lse_part, f32, (B, Hq, n_split), "lse_part"), _stream(stream)))
+
+
 def sas_decode_combine(p: Params, n_split: int, o_part, lse_part, o, lse_o=None, stream=None) -> None:
     B, Hq, d = p.batch, p.n_q_heads, p.head_dim
     _check("sas_decode_combine", lib.sas_decode_combine(
@@ -270,6 +287,15 @@ def prefill_step(p: Params, q, k, v, s, dO, out: dict, backward: bool = True, st
     if backward:
         sas_bwd(p, q, k, v, out["o"], dO, s, out["idx"], out["lse_s"], out["lse_o"], out["dq"], out["dk"], out["dv"],
                 out["ds"], out["ws"], stream=stream)
+
+
+def decode_step_paged(p: Params, q, k_pages, v_pages, block_table, cache_len, s, n_split: int, out: dict,
+                      stream=None) -> None:
+    """One decode step over a paged KV cache: select, split-K attention through the block table, merge."""
+    sas_topk_select(p, s, out["idx"], out["lse_s"], cache_len=cache_len, stream=stream)
+    sas_decode_paged(p, q, k_pages, v_pages, block_table, cache_len, s, out["idx"], out["lse_s"], n_split,
+                     out["o_part"], out["lse_part"], stream=stream)
+    sas_decode_combine(p, n_split, out["o_part"], out["lse_part"], out["o"], out["lse_o"], stream=stream)
 
 
 def decode_step(p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, stream=None) -> None:

@@ -16,6 +16,11 @@
 // memory before the ring starts, so no global load sits between two copies.
 // The ring uses only cp.async groups, with no spin-waits.
 //
+// The K/V arrays are either the dense cache [B, Hkv, Lmax, d] or a paged cache
+// [n_pages, Hkv, 64, d] with a block table: each task resolves its block to a
+// 64-row slice of the array when the task list is built, so the ring is the
+// same for both.
+//
 // The arithmetic runs on mma.sync, so that the instruction count stays below
 // the memory time. The G <= 8 query heads of a KV head are padded to one
 // 16-row A fragment that serves every K/V load (GQA grouping). Each warp
@@ -41,6 +46,8 @@ struct DecodeArgs {
   const float* s;
   const int32_t* idx;
   const float* lse_s;
+  const int32_t* table;  // paged cache: page of logical block m of sequence b at table[b * NB + m]; null if dense
+  int n_pages;
   float* o_part;
   float* lse_part;
   int* err;
@@ -57,7 +64,8 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
   constexpr int STAGEB = 2 * TILEB + QB;
   constexpr int DW = D / 4;             // d columns per warp in PV
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ int t_item[dec::kMaxTasks], t_m[dec::kMaxTasks], t_ntok[dec::kMaxTasks], t_flags[dec::kMaxTasks];
+  // per task: item, 64-row block of the K/V arrays (row b · 64), token count, first/last flags, gate
+  __shared__ int t_item[dec::kMaxTasks], t_blk[dec::kMaxTasks], t_ntok[dec::kMaxTasks], t_flags[dec::kMaxTasks];
   __shared__ float t_lam[dec::kMaxTasks];
   __shared__ int wsum_s[dec::kThreads / 32];
   __shared__ float red_max[4][8], red_sum[4][8];
@@ -153,8 +161,21 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
             lam = (a.s[size_t(bh) * NB + m] - lse_bh) * kLog2e;
           }
         }
+        int blk = bh * NB + m;  // dense cache [B, Hkv, Lmax, d]
+        if (a.table != nullptr) {  // paged cache [n_pages, Hkv, 64, d]
+          int pg = 0;
+          if (ntok > 0) {
+            const int b = bh / a.Hkv;
+            pg = a.table[size_t(b) * NB + m];
+            if (pg < 0 || pg >= a.n_pages) {
+              raise_error(a.err, SAS_ERR_DEVICE_INDEX);
+              pg = 0;
+            }
+          }
+          blk = pg * a.Hkv + bh % a.Hkv;
+        }
         t_item[base + j] = item;
-        t_m[base + j] = m;
+        t_blk[base + j] = blk;
         t_ntok[base + j] = ntok;
         t_lam[base + j] = lam;
         t_flags[base + j] = (j == 0 ? 1 : 0) | (j == cnt - 1 ? 2 : 0);
@@ -167,7 +188,7 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       const int it = t_item[task];
       const int bh = it / a.n_split;
       const int ntok = t_ntok[task];
-      const size_t row0 = size_t(bh) * a.Lmax + size_t(t_m[task]) * kBlock;
+      const size_t row0 = size_t(t_blk[task]) * kBlock;
       const uint16_t* kb = a.kc + row0 * D;
       const uint16_t* vb = a.vc + row0 * D;
       // rows past ntok are zero-filled (no bytes read), so masked tokens multiply finite zeros
@@ -386,9 +407,12 @@ static cudaError_t launch_decode_dg(const Shape& sh, const DecodeArgs& a, cudaSt
 
 template <int D>
 static cudaError_t launch_decode_d(const Shape& sh, const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
-                                   const int32_t* cl, const float* s, const int32_t* idx, const float* lse_s,
-                                   int n_split, float* o_part, float* lse_part, int* err, cudaStream_t st) {
+                                   const int32_t* table, int n_pages, const int32_t* cl, const float* s,
+                                   const int32_t* idx, const float* lse_s, int n_split, float* o_part,
+                                   float* lse_part, int* err, cudaStream_t st) {
   DecodeArgs a;
+  a.table = table;
+  a.n_pages = n_pages;
   a.q = q;
   a.kc = kc;
   a.vc = vc;
@@ -424,8 +448,18 @@ static cudaError_t launch_decode_d(const Shape& sh, const uint16_t* q, const uin
 cudaError_t launch_decode(const Shape& sh, const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                           const int32_t* cl, const float* s, const int32_t* idx, const float* lse_s, int n_split,
                           float* o_part, float* lse_part, int* err, cudaStream_t st) {
-  if (sh.d == 128) return launch_decode_d<128>(sh, q, kc, vc, cl, s, idx, lse_s, n_split, o_part, lse_part, err, st);
-  return launch_decode_d<64>(sh, q, kc, vc, cl, s, idx, lse_s, n_split, o_part, lse_part, err, st);
+  if (sh.d == 128)
+    return launch_decode_d<128>(sh, q, kc, vc, nullptr, 0, cl, s, idx, lse_s, n_split, o_part, lse_part, err, st);
+  return launch_decode_d<64>(sh, q, kc, vc, nullptr, 0, cl, s, idx, lse_s, n_split, o_part, lse_part, err, st);
+}
+
+cudaError_t launch_decode_paged(const Shape& sh, const uint16_t* q, const uint16_t* kp, const uint16_t* vp,
+                                int n_pages, const int32_t* table, const int32_t* cl, const float* s,
+                                const int32_t* idx, const float* lse_s, int n_split, float* o_part, float* lse_part,
+                                int* err, cudaStream_t st) {
+  if (sh.d == 128)
+    return launch_decode_d<128>(sh, q, kp, vp, table, n_pages, cl, s, idx, lse_s, n_split, o_part, lse_part, err, st);
+  return launch_decode_d<64>(sh, q, kp, vp, table, n_pages, cl, s, idx, lse_s, n_split, o_part, lse_part, err, st);
 }
 
 cudaError_t launch_decode_combine(const Shape& sh, int n_split, const float* o_part, const float* lse_part,

@@ -24,6 +24,10 @@ cudaError_t launch_bwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k
 cudaError_t launch_decode(const Shape& sh, const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                           const int32_t* cl, const float* s, const int32_t* idx, const float* lse_s, int n_split,
                           float* o_part, float* lse_part, int* err, cudaStream_t st);
+cudaError_t launch_decode_paged(const Shape& sh, const uint16_t* q, const uint16_t* kp, const uint16_t* vp,
+                                int n_pages, const int32_t* table, const int32_t* cl, const float* s,
+                                const int32_t* idx, const float* lse_s, int n_split, float* o_part, float* lse_part,
+                                int* err, cudaStream_t st);
 cudaError_t launch_decode_combine(const Shape& sh, int n_split, const float* o_part, const float* lse_part,
                                   uint16_t* o, float* lse_o, cudaStream_t st);
 }  // namespace sas
@@ -193,6 +197,25 @@ sas_status sas_decode(const sas_params* p, const sas_bf16* q, const sas_bf16* kc
   return from_cuda(sas::launch_decode(sh, q, kc, vc, cache_len, sh.gated ? s : nullptr, idx,
                                       sh.gated ? lse_s : nullptr, n_split, o_part, lse_part, device_error_word(),
                                       static_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_decode_paged(const sas_params* p, const sas_bf16* q, const sas_bf16* k_pages,
+                            const sas_bf16* v_pages, int n_pages, const int32_t* block_table,
+                            const int32_t* cache_len, const float* s, const int32_t* idx, const float* lse_s,
+                            int n_split, float* o_part, float* lse_part, void* stream) {
+  Shape sh;
+  sas_status r = make_shape(p, &sh);
+  if (r != SAS_OK) return r;
+  if (sh.G > 8) return SAS_ERR_UNSUPPORTED;
+  if (!ok_ptr(q) || !ok_ptr(k_pages) || !ok_ptr(v_pages) || !ok_ptr(block_table) || !ok_ptr(cache_len) ||
+      !ok_ptr(idx) || !ok_ptr(o_part) || !ok_ptr(lse_part))
+    return SAS_ERR_INVALID_ARG;
+  if (n_pages < 1 || int64_t(n_pages) * sh.Hkv > (int64_t(1) << 31) / sas::kBlock) return SAS_ERR_INVALID_ARG;
+  if (sh.gated && (!ok_ptr(s) || !ok_ptr(lse_s))) return SAS_ERR_INVALID_ARG;
+  if (n_split < 1 || n_split > sh.K + 1 || n_split > 65535) return SAS_ERR_INVALID_ARG;
+  return from_cuda(sas::launch_decode_paged(sh, q, k_pages, v_pages, n_pages, block_table, cache_len,
+                                            sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, n_split, o_part,
+                                            lse_part, device_error_word(), static_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_decode_combine(const sas_params* p, int n_split, const float* o_part, const float* lse_part,

@@ -40,6 +40,12 @@ were lost when the page was extracted):
 7. Decode: ``cache_len`` counts the new token. The current block is
    c = (L−1) // b and holds L − b·c tokens with gate 1. History is blocks
    0..c−1.
+8. Paged KV cache. [SAS-summary] §전제와 한계 measures decode inside a serving
+   engine, which keeps the cache in pages; the pages do not describe a
+   layout. A page here holds one block of every KV head, and a block table
+   maps logical blocks to pages. Paging changes where tokens are stored, not
+   what the step computes: ``decode_paged`` is ``decode`` on the gathered
+   dense cache.
 
 All arithmetic is float64. Inputs are taken as given; the generators round
 them to bf16 before either side sees them.
@@ -392,6 +398,42 @@ def decode(q, kc, vc, cache_len, s, K: int, block: int = 64, gate_mode: int = GA
                         q[b, hq], kc[b, h], vc[b, h], blist[a:e], L, s[b, h, :c], sel, gate_mode, scale, block)
     o, lse = decode_combine(o_part, lse_part)
     return dict(idx=idx, lse_s=lse_s, o_part=o_part, lse_part=lse_part, o=o, lse=lse)
+
+
+def gather_pages(k_pages, v_pages, block_table, cache_len, block: int = 64):
+    """Dense caches [B, Hkv, Lmax, d] from a paged cache.
+
+    A page holds one block of every KV head: k_pages and v_pages are
+    [n_pages, Hkv, block, d], and block_table[b, m] is the page of logical block
+    m of sequence b. Blocks 0..(L−1)/block of sequence b are copied. Everything
+    else stays zero, so a page's tokens past the cache length and the blocks
+    past the current one never enter the result.
+    """
+    k_pages = np.asarray(k_pages)
+    v_pages = np.asarray(v_pages)
+    B, NB = block_table.shape
+    _, Hkv, _, d = k_pages.shape
+    kc = np.zeros((B, Hkv, NB * block, d))
+    vc = np.zeros((B, Hkv, NB * block, d))
+    for b in range(B):
+        L = int(cache_len[b])
+        for m in range((L - 1) // block + 1):
+            n = min(block, L - m * block)  # tokens of block m that exist
+            pg = int(block_table[b, m])
+            kc[b, :, m * block:m * block + n] = k_pages[pg, :, :n]
+            vc[b, :, m * block:m * block + n] = v_pages[pg, :, :n]
+    return kc, vc
+
+
+def decode_paged(q, k_pages, v_pages, block_table, cache_len, s, K: int, block: int = 64,
+                 gate_mode: int = GATE_NONE, softmax_scale: Optional[float] = None, n_split: int = 1):
+    """Single-token decode over a paged KV cache.
+
+    The paged cache is only a storage layout. The step is the same decode as
+    ``decode``, over the dense cache that ``gather_pages`` rebuilds.
+    """
+    kc, vc = gather_pages(k_pages, v_pages, block_table, cache_len, block)
+    return decode(q, kc, vc, cache_len, s, K, block, gate_mode, softmax_scale, n_split)
 
 
 def decode_combine(o_part: np.ndarray, lse_part: np.ndarray):

@@ -137,3 +137,20 @@ def test_python_binding_refuses_cpu_tensors():
     idx = torch.zeros(1, 2, 2, 1, dtype=torch.int32)
     with pytest.raises(ValueError):
         sas.sas_topk_select(p, s, idx)
+
+
+def test_decode_paged_checked():
+    c = _p(top_k=4).c()
+
+    def call(n_pages=8, table=A, n_split=2, params=c):
+        # p, q, k_pages, v_pages, n_pages, block_table, cache_len, s, idx, lse_s, n_split, o_part, lse_part, stream
+        return lib.sas_decode_paged(ctypes.byref(params), A, A, A, n_pages, table, A, A, A, A, n_split, A, A, None)
+
+    assert call(n_pages=0) == INVALID
+    assert call(n_pages=-3) == INVALID
+    assert call(n_pages=1 << 30) == INVALID  # page rows would overflow a 32-bit row index
+    assert call(table=None) == INVALID
+    assert call(n_split=0) == INVALID
+    assert call(n_split=6) == INVALID  # > K + 1
+    c16 = _p(n_q_heads=32, n_kv_heads=2).c()  # G = 16: no decode kernel
+    assert call(params=c16) == UNSUPPORTED

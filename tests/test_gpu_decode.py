@@ -105,3 +105,70 @@ def test_decode_graph_replays_fresh_inputs():
         assert_idx_equal(out["idx"].cpu().numpy(), ref["idx"])
         assert max_abs(host(out["o"]), ref["o"]) < TOL_O
         assert max_abs(host(out["lse_o"]), ref["lse"]) < TOL_L
+
+
+def _paged(kc, vc, lens, g, n_extra=5):
+    """Pages [n_pages, Hkv, 64, d] holding each sequence's blocks 0..c at shuffled
+    slots, and the block table. Everything the step must not read is NaN (unused
+    pages, tokens past the cache length) or garbage (table entries past c)."""
+    B, Hkv, Lmax, d = kc.shape
+    NB = Lmax // 64
+    used = [(b, m) for b in range(B) for m in range((lens[b] - 1) // 64 + 1)]
+    n_pages = len(used) + n_extra
+    slots = g.permutation(n_pages)[: len(used)]
+    kp = np.full((n_pages, Hkv, 64, d), np.nan, np.float32)
+    vp = np.full((n_pages, Hkv, 64, d), np.nan, np.float32)
+    table = g.integers(-7, 3 * n_pages, size=(B, NB)).astype(np.int32)
+    for (b, m), pg in zip(used, slots):
+        n = min(64, lens[b] - 64 * m)
+        kp[pg, :, :n] = kc[b, :, 64 * m:64 * m + n]
+        vp[pg, :, :n] = vc[b, :, 64 * m:64 * m + n]
+        table[b, m] = pg
+    return kp, vp, table
+
+
+@pytest.mark.parametrize("gate", [O.GATE_NONE, O.GATE_LOG_SOFTMAX])
+@pytest.mark.parametrize("B,Hq,Hkv,d,Lmax,K,n_split,lens", [
+    (4, 32, 8, 128, 2048, 16, 17, [2048, 1, 1000, 1999]),
+    (3, 10, 2, 64, 1024, 4, 2, [64, 65, 1024]),
+])
+def test_decode_paged_parity(B, Hq, Hkv, d, Lmax, K, n_split, lens, gate):
+    """Decode through a block table over shuffled pages equals the oracle; NaN in
+    every page and token the step must not read never reaches the output."""
+    sas = _sas()
+    q, kc, vc, s = _case(B, Hq, Hkv, d, Lmax, seed=B * 7 + K)
+    g = np.random.default_rng(123 + K)
+    kp, vp, table = _paged(kc, vc, lens, g)
+    cl = np.array(lens, dtype=np.int32)
+    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=Lmax, top_k=K, gate_mode=gate)
+    out = sas.empty_decode_outputs(p, n_split)
+    sas.decode_step_paged(p, bf16_dev(q), bf16_dev(kp), bf16_dev(vp), torch.from_numpy(table).cuda(),
+                          torch.from_numpy(cl).cuda(), f32_dev(s), n_split, out)
+    torch.cuda.synchronize()
+    assert sas.sas_get_device_error() == 0
+    ref = O.decode_paged(q, kp, vp, table, cl, s.astype(np.float64), K, gate_mode=gate, n_split=n_split)
+    assert_idx_equal(out["idx"].cpu().numpy(), ref["idx"])
+    got = host(out["o"])
+    assert np.isfinite(got).all()
+    assert max_abs(got, ref["o"]) < TOL_O
+    assert max_abs(host(out["lse_o"]), ref["lse"]) < TOL_L
+
+
+def test_decode_paged_bad_page_is_reported():
+    """A table entry outside the page pool for a block the step reads raises the
+    device error word; the kernel reads page 0 instead and does not fault."""
+    sas = _sas()
+    B, Hq, Hkv, d, Lmax, K = 2, 8, 2, 128, 1024, 4
+    q, kc, vc, s = _case(B, Hq, Hkv, d, Lmax, seed=5)
+    g = np.random.default_rng(9)
+    lens = [700, 1024]
+    kp, vp, table = _paged(kc, vc, lens, g, n_extra=0)
+    table[1, (lens[1] - 1) // 64] = kp.shape[0] + 3  # the current block of sequence 1
+    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=Lmax, top_k=K,
+                   gate_mode=O.GATE_NONE)
+    out = sas.empty_decode_outputs(p, 2)
+    sas.decode_step_paged(p, bf16_dev(q), bf16_dev(kp), bf16_dev(vp), torch.from_numpy(table).cuda(),
+                          torch.tensor(lens, dtype=torch.int32).cuda(), f32_dev(s), 2, out)
+    torch.cuda.synchronize()
+    assert sas.sas_get_device_error() == 6  # SAS_ERR_DEVICE_INDEX
+    assert sas.sas_get_device_error() == 0  # read and cleared

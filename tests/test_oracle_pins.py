@@ -415,3 +415,58 @@ def test_combine_ignores_empty_splits():
     lse_part = np.array([[0.5, -np.inf, 0.5]])
     o, lse = O.decode_combine(o_part, lse_part)
     assert np.allclose(o, [[2.0, 0.5]]) and lse[0] == pytest.approx(0.5 + math.log(2))
+
+
+def _page_dense_cache(kc, vc, cl, blk, g, n_extra=3):
+    """Pages [n_pages, Hkv, blk, d] holding each sequence's blocks 0..c at shuffled
+    positions, and the block table. Unused pages, table entries past c and tokens
+    past each cache length are NaN or garbage: the step must never read them."""
+    B, Hkv, Lmax, d = kc.shape
+    NB = Lmax // blk
+    used = [(b, m) for b in range(B) for m in range((int(cl[b]) - 1) // blk + 1)]
+    n_pages = len(used) + n_extra
+    slots = g.permutation(n_pages)[: len(used)]
+    kp = np.full((n_pages, Hkv, blk, d), np.nan)
+    vp = np.full((n_pages, Hkv, blk, d), np.nan)
+    table = g.integers(-5, 10 * n_pages, size=(B, NB)).astype(np.int32)  # garbage outside 0..c
+    for (b, m), pg in zip(used, slots):
+        n = min(blk, int(cl[b]) - m * blk)
+        kp[pg, :, :n] = kc[b, :, m * blk:m * blk + n]
+        vp[pg, :, :n] = vc[b, :, m * blk:m * blk + n]
+        table[b, m] = pg
+    return kp, vp, table
+
+
+def test_paged_decode_is_attention_over_the_gathered_pages():
+    """Dense ungated K: plain attention of the last token over the tokens the pages
+    hold for its sequence, however the pages are laid out; NaN elsewhere is never read."""
+    blk, Lmax, d = 8, 64, 8
+    q, kc, vc, g = _decode_case(B=3, Hq=4, Hkv=2, Lmax=Lmax, d=d, seed=13)
+    cl = np.array([1, 30, 64], np.int32)
+    s = g.standard_normal((3, 2, Lmax // blk))
+    kp, vp, table = _page_dense_cache(kc, vc, cl, blk, g)
+    dec = O.decode_paged(q, kp, vp, table, cl, s, K=8, block=blk)
+    assert np.isfinite(dec["o"]).all()
+    for b in range(3):
+        L = cl[b]
+        for hq in range(4):
+            h = hq // 2
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[b, hq][None, None, None]), torch.from_numpy(kc[b, h, :L][None, None]),
+                torch.from_numpy(vc[b, h, :L][None, None])).numpy()[0, 0, 0]
+            assert np.abs(dec["o"][b, hq] - ref).max() < 1e-12
+
+
+@pytest.mark.parametrize("gate_mode", [O.GATE_NONE, O.GATE_LOG_SOFTMAX])
+def test_paged_decode_equals_dense_decode(gate_mode):
+    """Selection and gates too: the paged step gives the dense step's answer."""
+    blk, Lmax, d = 8, 96, 8
+    q, kc, vc, g = _decode_case(B=2, Hq=4, Hkv=2, Lmax=Lmax, d=d, seed=17)
+    cl = np.array([96, 53], np.int32)
+    s = g.standard_normal((2, 2, Lmax // blk))
+    kp, vp, table = _page_dense_cache(kc, vc, cl, blk, g)
+    ref = O.decode(q, kc, vc, cl, s, K=3, block=blk, gate_mode=gate_mode, n_split=2)
+    out = O.decode_paged(q, kp, vp, table, cl, s, K=3, block=blk, gate_mode=gate_mode, n_split=2)
+    assert (out["idx"] == ref["idx"]).all()
+    assert np.abs(out["o"] - ref["o"]).max() < 1e-12
+    assert np.abs(out["lse"] - ref["lse"]).max() < 1e-12
