@@ -75,7 +75,15 @@ typedef enum {
    * every token of selected history block m. The current block gets 0. */
   SAS_GATE_LOG_SOFTMAX = 0,
   /* Inference form (Algorithm 2): Top-K selection only, no gate term. */
-  SAS_GATE_NONE = 1
+  SAS_GATE_NONE = 1,
+  /* Ablations of the gate activation (SAS summary §무엇과 다른가: a sigmoid
+   * gate saturates to 1, unnormalised logits collapse to 0). Both stay inside
+   * the softmax in log form, like SAS_GATE_LOG_SOFTMAX, and need s but not
+   * lse_s (which may be NULL and is not read).
+   * log g_m = log σ(s_m): */
+  SAS_GATE_LOG_SIGMOID = 2,
+  /* log g_m = s_m: */
+  SAS_GATE_LOGIT = 3
 } sas_gate_mode;
 
 typedef struct {
@@ -124,15 +132,16 @@ SAS_API sas_status sas_gate_lse(const sas_params* p, const float* s, const int32
  * ------------------------------------------------------------------------- */
 
 /* o_i = Σ_{j∈S_t} softmax_j(z_ij) v_j with z_ij = scale·q_i·k_j + λ_j.
- * λ_j = s[t, m(j)] − lse_s[t] for tokens of the selected history blocks
- * (SAS_GATE_LOG_SOFTMAX) and 0 for the current block. In the current block,
- * column j is visible to row i only when j <= i.
+ * λ_j = log g_{m(j)} for tokens of the selected history blocks: s[t, m] −
+ * lse_s[t] (SAS_GATE_LOG_SOFTMAX), log σ(s[t, m]) (SAS_GATE_LOG_SIGMOID),
+ * s[t, m] (SAS_GATE_LOGIT) or 0 (SAS_GATE_NONE). λ is 0 for the current
+ * block. In the current block, column j is visible to row i only when j <= i.
  *   q      bf16 [B, Hq, N, d]
  *   k, v   bf16 [B, Hkv, N, d]
- *   s      fp32 [B, Hkv, NQB, NKB]. Read only under SAS_GATE_LOG_SOFTMAX.
+ *   s      fp32 [B, Hkv, NQB, NKB]. Read under every gate mode but SAS_GATE_NONE.
  *   idx    int32 [B, Hkv, NQB, K], as written by sas_topk_select.
  *   lse_s  fp32 [B, Hkv, NQB]. Required under SAS_GATE_LOG_SOFTMAX,
- *          ignored (may be NULL) under SAS_GATE_NONE.
+ *          ignored (may be NULL) under the other modes.
  *   o      bf16 [B, Hq, N, d]. Output.
  *   lse_o  fp32 [B, Hq, N]. Output, may be NULL. Row log-sum-exp of z,
  *          which the backward needs.
@@ -156,9 +165,11 @@ SAS_API sas_status sas_bwd_workspace_size(const sas_params* p, size_t* bytes);
  *   ds     fp32 [B, Hkv, NQB, NKB]. Output. With dl[t, m] the gradient for
  *          log g_m summed over block m's tokens, the rows of query block t and
  *          the G heads,
- *            ds[t, m] = dl[t, m]·[m ∈ I_t] − softmax(s[t, 0:t])_m · Σ_{m'∈I_t} dl[t, m'].
- *          Zero for m >= t, and zero everywhere under SAS_GATE_NONE. May be
- *          NULL under SAS_GATE_NONE.
+ *            ds[t, m] = dl[t, m]·[m ∈ I_t] − softmax(s[t, 0:t])_m · Σ_{m'∈I_t} dl[t, m']
+ *          under SAS_GATE_LOG_SOFTMAX, dl[t, m]·(1 − σ(s[t, m]))·[m ∈ I_t]
+ *          under SAS_GATE_LOG_SIGMOID and dl[t, m]·[m ∈ I_t] under
+ *          SAS_GATE_LOGIT. Zero for m >= t, and zero everywhere under
+ *          SAS_GATE_NONE. May be NULL under SAS_GATE_NONE.
  *   ws     device workspace of at least sas_bwd_workspace_size bytes,
  *          256-byte aligned. Its contents on entry do not matter. The call
  *          overwrites it.
@@ -178,7 +189,7 @@ SAS_API sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf1
 /* One new query token per sequence, at position L−1 with L = cache_len[b].
  * It attends to the current block c = (L−1)/b, whose tokens b·c..L−1 carry
  * gate 1, and to the selected history blocks idx[b, h, 0..n−1], n = min(K, c).
- * Under SAS_GATE_LOG_SOFTMAX those blocks get λ = s − lse_s. The ordered
+ * Under a gate mode those blocks get λ = log g (see sas_fwd). The ordered
  * block list [c, idx...] is cut into n_split contiguous chunks of
  * ceil((n+1)/n_split) blocks. Split j covers its chunk and writes that
  * chunk's normalised output and log-sum-exp. An empty chunk gives o = 0 and
@@ -186,9 +197,9 @@ SAS_API sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf1
  *   q          bf16 [B, Hq, d]
  *   kc, vc     bf16 [B, Hkv, Lmax, d]   (Lmax = seq_len)
  *   cache_len  int32 [B], 1 <= L <= Lmax
- *   s          fp32 [B, Hkv, NKB]. Read only under SAS_GATE_LOG_SOFTMAX.
+ *   s          fp32 [B, Hkv, NKB]. Read under every gate mode but SAS_GATE_NONE.
  *   idx        int32 [B, Hkv, K] from sas_topk_select (decode form)
- *   lse_s      fp32 [B, Hkv]. Required under SAS_GATE_LOG_SOFTMAX.
+ *   lse_s      fp32 [B, Hkv]. Required under SAS_GATE_LOG_SOFTMAX only.
  *   n_split    1..K+1
  *   o_part     fp32 [B, Hq, n_split, d]. Output.
  *   lse_part   fp32 [B, Hq, n_split]. Output. */

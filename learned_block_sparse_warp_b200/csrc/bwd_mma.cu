@@ -170,7 +170,7 @@ __global__ void revidx_scan_kernel(const int* __restrict__ cnt, int NB, int* __r
 __global__ void __launch_bounds__(256) revidx_fill_kernel(const int32_t* __restrict__ idx, int nbh, int NB, int K,
                                                           const int* __restrict__ off, int* __restrict__ list,
                                                           const float* __restrict__ s, const float* __restrict__ lse_s,
-                                                          int gated, float* __restrict__ lam) {
+                                                          int gate, float* __restrict__ lam) {
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (w >= nbh * NB) return;
   const int lane = threadIdx.x & 31;
@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const int32_t* __restr
       out[at] = (t << 8) | slot;
       if (lam != nullptr) {  // the gate of block j for query block t, log2 domain
         const size_t row = size_t(bh) * NB + t;
-        lam[size_t(bh) * NB * K + at] = gated ? (s[row * NB + j] - lse_s[row]) * kLog2e : 0.f;
+        lam[size_t(bh) * NB * K + at] =
+            gate != SAS_GATE_NONE ? gate_lam2(gate, s[row * NB + j], lse_s != nullptr ? lse_s[row] : 0.f) : 0.f;
       }
     }
     pos += __popc(mask);
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(256, 1) bwd_main_kernel(
     float lam2 = 0.f;
     if (!diag && sh.gated) {
       const size_t row = bh * sh.NB + t;
-      lam2 = (s[row * sh.NB + j] - lse_s[row]) * kLog2e;
+      lam2 = gate_lam2(sh.gate, s[row * sh.NB + j], lse_s != nullptr ? lse_s[row] : 0.f);
     }
     const uint32_t cQ = sQ + stage * TILE, cdO = sdO + stage * TILE;
 
@@ -445,32 +446,39 @@ __global__ void bwd_dq_convert_kernel(const float4* __restrict__ acc, size_t n4,
 __global__ void __launch_bounds__(256) bwd_ds_chain_kernel(const float* __restrict__ s, const float* __restrict__ lse_s,
                                                            const int32_t* __restrict__ idx,
                                                            const float* __restrict__ dl, int rows, int NB, int K,
-                                                           int gated, float* __restrict__ ds) {
+                                                           int gate, float* __restrict__ ds) {
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (r >= rows) return;
   const int lane = threadIdx.x & 31;
   const int t = r % NB;
   float* dsr = ds + size_t(r) * NB;
-  if (!gated || t == 0) {
+  if (gate == SAS_GATE_NONE || t == 0) {
     for (int m = lane; m < NB; m += 32) dsr[m] = 0.f;
     return;
   }
   const int n = min(K, t);
   const int32_t* ir = idx + size_t(r) * K;
   const float* dlr = dl + size_t(r) * K;
-  float sum = 0.f;
-  for (int kk = lane; kk < n; kk += 32) {
-    const int m = ir[kk];
-    if (m >= 0 && m < t) sum += dlr[kk];
-  }
-  sum = warp_sum(sum);
-  const float lse = lse_s[r];
   const float* sr = s + size_t(r) * NB;
-  for (int m = lane; m < NB; m += 32) dsr[m] = (m < t) ? -expf(sr[m] - lse) * sum : 0.f;
+  if (gate == SAS_GATE_LOG_SOFTMAX) {  // every history block couples through LSE(s)
+    float sum = 0.f;
+    for (int kk = lane; kk < n; kk += 32) {
+      const int m = ir[kk];
+      if (m >= 0 && m < t) sum += dlr[kk];
+    }
+    sum = warp_sum(sum);
+    const float lse = lse_s[r];
+    for (int m = lane; m < NB; m += 32) dsr[m] = (m < t) ? -expf(sr[m] - lse) * sum : 0.f;
+  } else {  // log σ(s) and the raw logit act on each selected block alone
+    for (int m = lane; m < NB; m += 32) dsr[m] = 0.f;
+  }
   __syncwarp();
   for (int kk = lane; kk < n; kk += 32) {
     const int m = ir[kk];
-    if (m >= 0 && m < t) dsr[m] += dlr[kk];
+    if (m < 0 || m >= t) continue;
+    float x = dlr[kk];
+    if (gate == SAS_GATE_LOG_SIGMOID) x *= 1.f / (1.f + expf(sr[m]));  // d log σ(s) / ds = 1 − σ(s) = σ(−s)
+    dsr[m] += x;
   }
 }
 
@@ -504,7 +512,7 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
   revidx_count_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_cnt);
   revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
   revidx_fill_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_off, ws.rev_list, s, lse_s,
-                                                    sh.gated, D == 128 ? ws.rev_lam : nullptr);
+                                                    sh.gate, D == 128 ? ws.rev_lam : nullptr);
   if (D == 128) {  // tcgen05 passes: dK/dV/dl KV-major, then dQ query-major; no dQ accumulator
     if ((e = launch_bwd_passes_sm100(sh, q, k, v, dO, s, idx, lse_s, lse_o, ws.drow, ws.rev_off, ws.rev_list,
                                      ws.rev_lam, ws.dl,
@@ -512,7 +520,7 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
       return e;
     if (ds != nullptr) {
       const int rows = nbh * sh.NB;
-      bwd_ds_chain_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, lse_s, idx, ws.dl, rows, sh.NB, sh.K, sh.gated, ds);
+      bwd_ds_chain_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, lse_s, idx, ws.dl, rows, sh.NB, sh.K, sh.gate, ds);
     }
     return cudaGetLastError();
   }
@@ -528,7 +536,7 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
                                                   reinterpret_cast<uint2*>(dq));
   if (ds != nullptr) {
     const int rows = nbh * sh.NB;
-    bwd_ds_chain_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, lse_s, idx, ws.dl, rows, sh.NB, sh.K, sh.gated, ds);
+    bwd_ds_chain_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, lse_s, idx, ws.dl, rows, sh.NB, sh.K, sh.gate, ds);
   }
   return cudaGetLastError();
 }

@@ -42,7 +42,7 @@ struct BwdSm100Args {
   uint16_t* dv;
   const int32_t* idx;
   int* err;
-  int B, Hq, Hkv, G, N, NB, K, gated, n_hp, n_tp;
+  int B, Hq, Hkv, G, N, NB, K, gate, gated, n_hp, n_tp;
   float scale;
 };
 
@@ -539,7 +539,7 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
   if (warp == 0) {
     const size_t row = bh * a.NB + t;
     build_block_list(a.idx + row * a.K, a.K, t, a.gated ? a.s + row * a.NB : nullptr,
-                     a.gated ? a.lse_s[row] : 0.f, a.gated, list_s, lam_s, &nlist_s, a.err);
+                     a.lse_s != nullptr ? a.lse_s[row] : 0.f, a.gate, list_s, lam_s, &nlist_s, a.err);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&tmem_s), 512);
@@ -794,6 +794,7 @@ cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const ui
   a.N = sh.N;
   a.NB = sh.NB;
   a.K = sh.K;
+  a.gate = sh.gate;
   a.gated = sh.gated;
   a.n_hp = (sh.G + 1) / 2;
   a.n_tp = (sh.G + 3) / 4;

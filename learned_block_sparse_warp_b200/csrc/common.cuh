@@ -20,8 +20,20 @@ constexpr float kLn2 = 0.6931471805599453f;
 struct Shape {
   int B, Hq, Hkv, G, d, N, NB, K;
   float scale;  // softmax scale (1/sqrt(d) unless given)
-  int gated;    // 1 = log-softmax gate inside the softmax, 0 = no gate
+  int gate;     // sas_gate_mode
+  int gated;    // 1 when the gate puts a log g inside the softmax (every mode but SAS_GATE_NONE)
 };
+
+// λ_m of a selected history block in log2 units, log g_m · log2 e, for the gate
+// mode: s_m − LSE(s) (softmax-normalised), log σ(s_m), s_m (raw logit), or 0.
+__device__ __forceinline__ float gate_lam2(int gate, float s_m, float lse) {
+  switch (gate) {
+    case SAS_GATE_LOG_SOFTMAX: return (s_m - lse) * kLog2e;
+    case SAS_GATE_LOG_SIGMOID: return (fminf(s_m, 0.f) - log1pf(expf(-fabsf(s_m)))) * kLog2e;
+    case SAS_GATE_LOGIT: return s_m * kLog2e;
+    default: return 0.f;
+  }
+}
 
 // First error wins. The word lives in device memory owned by the library
 // (one per device) and is read back by sas_get_device_error.
@@ -123,7 +135,7 @@ __device__ __forceinline__ uint32_t score_key(float x) {
 // Builds the ordered block list [t, I_t...] of one query block in shared
 // memory with each block's log2-domain gate. Run by one warp.
 __device__ __forceinline__ void build_block_list(const int32_t* __restrict__ idx_row, int K, int t,
-                                                 const float* __restrict__ s_row, float lse_t, int gated,
+                                                 const float* __restrict__ s_row, float lse_t, int gate,
                                                  int* list_s, float* lam_s, int* nlist_s, int* err) {
   const int lane = threadIdx.x & 31;
   const int n = min(K, t);
@@ -142,7 +154,7 @@ __device__ __forceinline__ void build_block_list(const int32_t* __restrict__ idx
     if (ok) {
       const int pos = 1 + cnt + __popc(ok_mask & ((1u << lane) - 1u));
       list_s[pos] = m;
-      lam_s[pos] = gated ? (s_row[m] - lse_t) * kLog2e : 0.f;
+      lam_s[pos] = gate != SAS_GATE_NONE ? gate_lam2(gate, s_row[m], lse_t) : 0.f;
     }
     cnt += __popc(ok_mask);
     stop = end_mask != 0;

@@ -51,7 +51,7 @@ struct DecodeArgs {
   float* o_part;
   float* lse_part;
   int* err;
-  int B, Hkv, Lmax, K, gated, n_split, per_max, items_per_chunk;
+  int B, Hkv, Lmax, K, gate, gated, n_split, per_max, items_per_chunk;
   float scale;
 };
 
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
             m = 0;
             ntok = 0;  // an empty block
           } else if (a.gated) {
-            lam = (a.s[size_t(bh) * NB + m] - lse_bh) * kLog2e;
+            lam = gate_lam2(a.gate, a.s[size_t(bh) * NB + m], lse_bh);
           }
         }
         int blk = bh * NB + m;  // dense cache [B, Hkv, Lmax, d]
@@ -427,6 +427,7 @@ static cudaError_t launch_decode_d(const Shape& sh, const uint16_t* q, const uin
   a.Hkv = sh.Hkv;
   a.Lmax = sh.N;
   a.K = sh.K;
+  a.gate = sh.gate;
   a.gated = sh.gated;
   a.n_split = n_split;
   a.per_max = (sh.K + 1 + n_split - 1) / n_split;

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(128) fwd_mma_kernel(const uint16_t* __restrict
   if (warp == 0) {
     const size_t row = bh * sh.NB + t;
     build_block_list(idx + row * sh.K, sh.K, t, sh.gated ? s + row * sh.NB : nullptr,
-                     sh.gated ? lse_s[row] : 0.f, sh.gated, list_s, lam_s, &nlist_s, err);
+                     lse_s != nullptr ? lse_s[row] : 0.f, sh.gate, list_s, lam_s, &nlist_s, err);
   }
   const uint16_t* qg = q + ((size_t(b) * sh.Hq + hq) * sh.N + size_t(t) * kBlock) * D;
   const uint16_t* kg = k + bh * size_t(sh.N) * D;

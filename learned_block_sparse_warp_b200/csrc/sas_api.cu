@@ -63,13 +63,21 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 
+// Gate inputs: s for every gate mode but SAS_GATE_NONE, and lse_s for the
+// softmax-normalised gate. The ablation modes do not read lse_s (it may be NULL).
+bool gate_inputs_ok(const Shape& sh, const float* s, const float* lse_s) {
+  if (!sh.gated) return true;
+  if (!ok_ptr(s) || !ok_opt(lse_s)) return false;
+  return sh.gate != SAS_GATE_LOG_SOFTMAX || lse_s != nullptr;
+}
+
 // Checks the shared parameters and fills the kernel-side shape.
 sas_status make_shape(const sas_params* p, Shape* sh) {
   if (p == nullptr) return SAS_ERR_INVALID_ARG;
   if (p->batch < 1 || p->n_q_heads < 1 || p->n_kv_heads < 1 || p->seq_len < 1 || p->top_k < 1)
     return SAS_ERR_INVALID_ARG;
   if (p->n_q_heads % p->n_kv_heads != 0) return SAS_ERR_INVALID_ARG;
-  if (p->gate_mode != SAS_GATE_LOG_SOFTMAX && p->gate_mode != SAS_GATE_NONE) return SAS_ERR_INVALID_ARG;
+  if (p->gate_mode < SAS_GATE_LOG_SOFTMAX || p->gate_mode > SAS_GATE_LOGIT) return SAS_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.f) || isinf(p->softmax_scale)) return SAS_ERR_INVALID_ARG;
   if (p->top_k > sas::kMaxTopK) return SAS_ERR_INVALID_ARG;
   if (p->block != sas::kBlock) return SAS_ERR_UNSUPPORTED;
@@ -88,7 +96,8 @@ sas_status make_shape(const sas_params* p, Shape* sh) {
   sh->NB = int(nb);
   sh->K = p->top_k;
   sh->scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(float(p->head_dim));
-  sh->gated = p->gate_mode == SAS_GATE_LOG_SOFTMAX ? 1 : 0;
+  sh->gate = p->gate_mode;
+  sh->gated = p->gate_mode != SAS_GATE_NONE ? 1 : 0;
   return SAS_OK;
 }
 
@@ -146,7 +155,7 @@ sas_status sas_fwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, co
   if (r != SAS_OK) return r;
   if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(idx) || !ok_ptr(o) || !ok_opt(lse_o))
     return SAS_ERR_INVALID_ARG;
-  if (sh.gated && (!ok_ptr(s) || !ok_ptr(lse_s))) return SAS_ERR_INVALID_ARG;
+  if (!gate_inputs_ok(sh, s, lse_s)) return SAS_ERR_INVALID_ARG;
   // d = 128: TMA + tcgen05 kernel; d = 64: warp-level tensor-core kernel
   if (sh.d == 128)
     return from_cuda(sas::launch_fwd_sm100(sh, q, k, v, sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, o,
@@ -173,7 +182,7 @@ sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, co
   if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) || !ok_ptr(dO) || !ok_ptr(idx) || !ok_ptr(lse_o) ||
       !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv))
     return SAS_ERR_INVALID_ARG;
-  if (sh.gated && (!ok_ptr(s) || !ok_ptr(lse_s) || !ok_ptr(ds))) return SAS_ERR_INVALID_ARG;
+  if (!gate_inputs_ok(sh, s, lse_s) || (sh.gated && !ok_ptr(ds))) return SAS_ERR_INVALID_ARG;
   if (!ok_opt(ds)) return SAS_ERR_INVALID_ARG;
   const size_t need = sas::bwd_ws_layout(sh, nullptr, nullptr);
   if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SAS_ERR_WORKSPACE;
@@ -192,7 +201,7 @@ sas_status sas_decode(const sas_params* p, const sas_bf16* q, const sas_bf16* kc
   if (!ok_ptr(q) || !ok_ptr(kc) || !ok_ptr(vc) || !ok_ptr(cache_len) || !ok_ptr(idx) || !ok_ptr(o_part) ||
       !ok_ptr(lse_part))
     return SAS_ERR_INVALID_ARG;
-  if (sh.gated && (!ok_ptr(s) || !ok_ptr(lse_s))) return SAS_ERR_INVALID_ARG;
+  if (!gate_inputs_ok(sh, s, lse_s)) return SAS_ERR_INVALID_ARG;
   if (n_split < 1 || n_split > sh.K + 1 || n_split > 65535) return SAS_ERR_INVALID_ARG;
   return from_cuda(sas::launch_decode(sh, q, kc, vc, cache_len, sh.gated ? s : nullptr, idx,
                                       sh.gated ? lse_s : nullptr, n_split, o_part, lse_part, device_error_word(),
@@ -211,7 +220,7 @@ sas_status sas_decode_paged(const sas_params* p, const sas_bf16* q, const sas_bf
       !ok_ptr(idx) || !ok_ptr(o_part) || !ok_ptr(lse_part))
     return SAS_ERR_INVALID_ARG;
   if (n_pages < 1 || int64_t(n_pages) * sh.Hkv > (int64_t(1) << 31) / sas::kBlock) return SAS_ERR_INVALID_ARG;
-  if (sh.gated && (!ok_ptr(s) || !ok_ptr(lse_s))) return SAS_ERR_INVALID_ARG;
+  if (!gate_inputs_ok(sh, s, lse_s)) return SAS_ERR_INVALID_ARG;
   if (n_split < 1 || n_split > sh.K + 1 || n_split > 65535) return SAS_ERR_INVALID_ARG;
   return from_cuda(sas::launch_decode_paged(sh, q, k_pages, v_pages, n_pages, block_table, cache_len,
                                             sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, n_split, o_part,

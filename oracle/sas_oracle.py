@@ -59,6 +59,11 @@ import numpy as np
 
 GATE_LOG_SOFTMAX = 0  # training form, Eq. (9)
 GATE_NONE = 1  # inference form (Algorithm 2): Top-K only, no gate
+# Ablations of the gate activation ([SAS-summary] §무엇과 다른가): a sigmoid gate,
+# which saturates to 1, and the raw logit injected unnormalised, which collapses
+# to 0. Both stay inside the softmax in log form.
+GATE_LOG_SIGMOID = 2  # log g_m = log σ(s_m)
+GATE_LOGIT = 3  # log g_m = s_m
 
 
 def _scale(d: int, softmax_scale: Optional[float]) -> float:
@@ -135,12 +140,39 @@ def decode_select(s: np.ndarray, cache_len: np.ndarray, K: int, block: int = 64)
 # [SAS-explainer] §仕組み: g0 = 1 for B0, one value per block broadcast to its
 # tokens)
 # ---------------------------------------------------------------------------
+def _log_sigmoid(x: float) -> float:
+    """log σ(x) = −log(1 + e^(−x)), written so that neither branch overflows."""
+    return -math.log1p(math.exp(-x)) if x >= 0 else x - math.log1p(math.exp(x))
+
+
 def log_gate(s_hist: np.ndarray, selected: Sequence[int], gate_mode: int) -> np.ndarray:
     """log g_m for the selected history blocks (0 for every block under GATE_NONE)."""
     if gate_mode == GATE_NONE:
         return np.zeros(len(selected))
+    if gate_mode == GATE_LOG_SIGMOID:
+        return np.array([_log_sigmoid(float(s_hist[m])) for m in selected], dtype=np.float64)
+    if gate_mode == GATE_LOGIT:
+        return np.array([float(s_hist[m]) for m in selected], dtype=np.float64)
     lse = logsumexp(s_hist)
     return np.array([float(s_hist[m]) - lse for m in selected], dtype=np.float64)
+
+
+def gate_score_gradient(s_hist: np.ndarray, selected: Sequence[int], dl_sel: np.ndarray, gate_mode: int) -> np.ndarray:
+    """ds over the history blocks from dl = ∂loss/∂log g of the selected ones.
+
+    log-softmax: ds_m = dl_m·[m ∈ I] − softmax(s)_m Σ dl (every history block
+    couples through LSE). log-sigmoid: ds_m = dl_m (1 − σ(s_m)) on the selected
+    blocks. logit: ds_m = dl_m on the selected blocks.
+    """
+    sh = np.asarray(s_hist, np.float64)
+    ds_row = np.zeros(len(sh))
+    if gate_mode == GATE_LOG_SOFTMAX:
+        ds_row = -np.exp(sh - logsumexp(sh)) * float(np.sum(dl_sel))
+    for m, x in zip(selected, dl_sel):
+        if gate_mode == GATE_LOG_SIGMOID:
+            x = x * (1.0 - 1.0 / (1.0 + math.exp(-sh[m])))
+        ds_row[m] += x
+    return ds_row
 
 
 def _gathered_tokens(t: int, selected: Sequence[int], block: int, n_cur: int) -> np.ndarray:
@@ -221,7 +253,8 @@ def backward(q, k, v, s, idx, do, block: int = 64, gate_mode: int = GATE_LOG_SOF
     Returns dq [B, Hq, N, d], dk, dv [B, Hkv, N, d], ds [B, Hkv, NQB, NKB] and
     dl [B, Hkv, NQB, K]. dl[t, slot] is the gradient with respect to log g of the
     block idx[t, slot], summed over the block's tokens, the query block's rows and
-    the group's heads. ds follows from log g_m = s_m − LSE(s):
+    the group's heads. ds follows from log g_m(s) of the gate mode (see
+    ``gate_score_gradient``); for the softmax-normalised gate,
     ds_m = dl_m·[m ∈ I] − softmax(s)_m Σ_{m'∈I} dl_m'.
 
     ``o`` (the forward output) is recomputed when not given. With ``t_list`` only
@@ -273,13 +306,8 @@ def backward(q, k, v, s, idx, do, block: int = 64, gate_mode: int = GATE_LOG_SOF
                     continue
                 dl_sel = dlam_tok[block:].reshape(len(sel), block).sum(axis=1)
                 dl[b, h, t, : len(sel)] = dl_sel
-                # chain through log g_m = s_m − LSE(s_hist)
-                sh = np.asarray(s[b, h, t, :t], np.float64)
-                soft = np.exp(sh - logsumexp(sh))
-                ds_row = -soft * dl_sel.sum()
-                for m, x in zip(sel, dl_sel):
-                    ds_row[m] += x
-                ds[b, h, t, :t] = ds_row
+                # chain through log g_m(s_hist) of the gate mode
+                ds[b, h, t, :t] = gate_score_gradient(s[b, h, t, :t], sel, dl_sel, gate_mode)
     return dq, dk, dv, ds, dl
 
 

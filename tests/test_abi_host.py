@@ -154,3 +154,13 @@ def test_decode_paged_checked():
     assert call(n_split=6) == INVALID  # > K + 1
     c16 = _p(n_q_heads=32, n_kv_heads=2).c()  # G = 16: no decode kernel
     assert call(params=c16) == UNSUPPORTED
+
+
+def test_gate_ablation_inputs_checked():
+    # the ablations read s but not lse_s: s is required, lse_s may be NULL
+    for mode in (2, 3):
+        assert _fwd(_p(gate_mode=mode), s=None) == INVALID
+    assert _fwd(_p(gate_mode=0), lse_s=None) == INVALID
+    assert _fwd(_p(gate_mode=4)) == INVALID
+    c = _p(gate_mode=2).c()
+    assert lib.sas_decode(ctypes.byref(c), A, A, A, A, None, A, None, 2, A, A, None) == INVALID  # s missing

@@ -4,7 +4,7 @@ import pytest
 
 import oracle.sas_oracle as O
 from synth import workloads as W
-from tests.parity_util import TOL_REL, assert_idx_equal, rel_fro
+from tests.parity_util import TOL_L, TOL_O, TOL_REL, assert_idx_equal, max_abs, rel_fro
 from tests.test_gpu_fwd import run_prefill
 
 pytestmark = pytest.mark.gpu
@@ -25,9 +25,28 @@ CASES = [
 ]
 
 
+ABLATION_CASES = [c for c in CASES if c[0] in ("tiny", "gqa4_d128", "g3_d128_k1", "g2_d128_b2")]
+
+
 @pytest.mark.parametrize("gate", [O.GATE_LOG_SOFTMAX, O.GATE_NONE])
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_bwd_parity(case, gate):
+    _check_bwd(case, gate)
+
+
+@pytest.mark.parametrize("gate", [O.GATE_LOG_SIGMOID, O.GATE_LOGIT])
+@pytest.mark.parametrize("case", ABLATION_CASES, ids=[c[0] for c in ABLATION_CASES])
+def test_bwd_gate_ablations(case, gate):
+    """The gate-activation ablations: log σ(s) and the raw logit inside the softmax,
+    with their own chain to ds. The forward output is checked on the way."""
+    x, r = _check_bwd(case, gate)
+    ref_idx, _ = O.prefill_select(x["s"].astype(np.float64), case[6])
+    o, L = O.forward(x["q"], x["k"], x["v"], x["s"], ref_idx, gate_mode=gate)
+    assert max_abs(r["o"], o) < TOL_O
+    assert max_abs(r["lse_o"], L) < TOL_L
+
+
+def _check_bwd(case, gate):
     name, B, Hq, Hkv, d, N, K = case
     w = W.custom(name, batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=N, top_k=K, seed=200 + len(name))
     x, r, err = run_prefill(w, gate, backward=True)
@@ -48,6 +67,7 @@ def test_bwd_parity(case, gate):
         assert np.all(r["ds"][..., iu[0], iu[1]] == 0)
     else:
         assert np.all(r["ds"] == 0)
+    return x, r
 
 
 def test_bwd_tiny_workload_exact_config():

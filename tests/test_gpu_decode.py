@@ -172,3 +172,25 @@ def test_decode_paged_bad_page_is_reported():
     torch.cuda.synchronize()
     assert sas.sas_get_device_error() == 6  # SAS_ERR_DEVICE_INDEX
     assert sas.sas_get_device_error() == 0  # read and cleared
+
+
+@pytest.mark.parametrize("gate", [O.GATE_LOG_SIGMOID, O.GATE_LOGIT])
+def test_decode_gate_ablations(gate):
+    """Decode under the gate-activation ablations (lse_s is not needed and not passed)."""
+    sas = _sas()
+    B, Hq, Hkv, d, Lmax, K, n_split = 3, 16, 4, 128, 2048, 8, 3
+    q, kc, vc, s = _case(B, Hq, Hkv, d, Lmax, seed=61)
+    lens = [2048, 777, 65]
+    cl = np.array(lens, dtype=np.int32)
+    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=Lmax, top_k=K, gate_mode=gate)
+    out = sas.empty_decode_outputs(p, n_split)
+    qd, kd, vd, sd, cld = bf16_dev(q), bf16_dev(kc), bf16_dev(vc), f32_dev(s), torch.from_numpy(cl).cuda()
+    sas.sas_topk_select(p, sd, out["idx"], None, cache_len=cld)
+    sas.sas_decode(p, qd, kd, vd, cld, sd, out["idx"], None, n_split, out["o_part"], out["lse_part"])
+    sas.sas_decode_combine(p, n_split, out["o_part"], out["lse_part"], out["o"], out["lse_o"])
+    torch.cuda.synchronize()
+    assert sas.sas_get_device_error() == 0
+    ref = O.decode(q, kc, vc, cl, s.astype(np.float64), K, gate_mode=gate, n_split=n_split)
+    assert_idx_equal(out["idx"].cpu().numpy(), ref["idx"])
+    assert max_abs(host(out["o"]), ref["o"]) < TOL_O
+    assert max_abs(host(out["lse_o"]), ref["lse"]) < TOL_L

@@ -287,7 +287,7 @@ def test_gate_reweights_probabilities():
 # ---------------------------------------------------------------------------
 # Gradients: central finite differences and the pages' gate-gradient formula
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("gate_mode", [O.GATE_LOG_SOFTMAX, O.GATE_NONE])
+@pytest.mark.parametrize("gate_mode", [O.GATE_LOG_SOFTMAX, O.GATE_NONE, O.GATE_LOG_SIGMOID, O.GATE_LOGIT])
 def test_gradients_finite_differences(gate_mode):
     blk, N, d, K = 4, 16, 4, 2
     q, k, v, do, s = _rand_case(B=1, Hq=2, Hkv=1, N=N, d=d, block=blk, seed=31, s_spread=True)
@@ -470,3 +470,20 @@ def test_paged_decode_equals_dense_decode(gate_mode):
     assert (out["idx"] == ref["idx"]).all()
     assert np.abs(out["o"] - ref["o"]).max() < 1e-12
     assert np.abs(out["lse"] - ref["lse"]).max() < 1e-12
+
+
+
+def test_gate_ablations_have_their_closed_forms():
+    """log σ and the raw logit, as the gate-activation ablations define them, for
+    scores far into both tails; the selected set does not matter for either."""
+    s_hist = np.array([-40.0, -3.0, 0.0, 2.5, 40.0])
+    sel = [0, 1, 2, 3, 4]
+    ls = O.log_gate(s_hist, sel, O.GATE_LOG_SIGMOID)
+    ref = -np.logaddexp(0.0, -s_hist)  # log σ(x) = −log(1 + e^(−x))
+    assert np.abs(ls - ref).max() < 1e-14
+    assert O.log_gate(s_hist, sel, O.GATE_LOGIT).tolist() == s_hist.tolist()
+    # the softmax-normalised gate is invariant to a global shift of the scores; the ablations are not
+    for mode, inv in ((O.GATE_LOG_SOFTMAX, True), (O.GATE_LOG_SIGMOID, False), (O.GATE_LOGIT, False)):
+        a = O.log_gate(s_hist[1:4], [0, 2], mode)
+        b = O.log_gate(s_hist[1:4] + 1.5, [0, 2], mode)
+        assert (np.abs(a - b).max() < 1e-12) == inv
