@@ -200,7 +200,8 @@ SAS_API sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf1
  *   s          fp32 [B, Hkv, NKB]. Read under every gate mode but SAS_GATE_NONE.
  *   idx        int32 [B, Hkv, K] from sas_topk_select (decode form)
  *   lse_s      fp32 [B, Hkv]. Required under SAS_GATE_LOG_SOFTMAX only.
- *   n_split    1..K+1
+ *   n_split    1..K+1, with ceil((K+1) / n_split) <= 64 (SAS_ERR_UNSUPPORTED
+ *              otherwise): a split covers at most 64 blocks.
  *   o_part     fp32 [B, Hq, n_split, d]. Output.
  *   lse_part   fp32 [B, Hq, n_split]. Output. */
 SAS_API sas_status sas_decode(const sas_params* p, const sas_bf16* q, const sas_bf16* kc, const sas_bf16* vc,

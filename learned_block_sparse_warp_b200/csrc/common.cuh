@@ -13,6 +13,7 @@ namespace sas {
 
 constexpr int kBlock = 64;          // tokens per block (b)
 constexpr int kMaxTopK = 256;       // largest K the kernels accept
+constexpr int kMaxDecodeBlocksPerSplit = 64;  // ceil((K + 1) / n_split) fits the decode task list
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

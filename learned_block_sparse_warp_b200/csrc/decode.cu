@@ -35,7 +35,7 @@ namespace sas {
 
 namespace dec {
 constexpr int kThreads = 128;
-constexpr int kMaxTasks = 64;   // task slots per chunk of items (keeps 2 CTAs per SM at d = 128)
+constexpr int kMaxTasks = kMaxDecodeBlocksPerSplit;  // task slots per chunk of items (2 CTAs per SM at d = 128)
 }  // namespace dec
 
 struct DecodeArgs {

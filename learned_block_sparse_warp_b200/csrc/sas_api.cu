@@ -203,6 +203,7 @@ sas_status sas_decode(const sas_params* p, const sas_bf16* q, const sas_bf16* kc
     return SAS_ERR_INVALID_ARG;
   if (!gate_inputs_ok(sh, s, lse_s)) return SAS_ERR_INVALID_ARG;
   if (n_split < 1 || n_split > sh.K + 1 || n_split > 65535) return SAS_ERR_INVALID_ARG;
+  if ((sh.K + n_split) / n_split > sas::kMaxDecodeBlocksPerSplit) return SAS_ERR_UNSUPPORTED;
   return from_cuda(sas::launch_decode(sh, q, kc, vc, cache_len, sh.gated ? s : nullptr, idx,
                                       sh.gated ? lse_s : nullptr, n_split, o_part, lse_part, device_error_word(),
                                       static_cast<cudaStream_t>(stream)));
@@ -222,6 +223,7 @@ sas_status sas_decode_paged(const sas_params* p, const sas_bf16* q, const sas_bf
   if (n_pages < 1 || int64_t(n_pages) * sh.Hkv > (int64_t(1) << 31) / sas::kBlock) return SAS_ERR_INVALID_ARG;
   if (!gate_inputs_ok(sh, s, lse_s)) return SAS_ERR_INVALID_ARG;
   if (n_split < 1 || n_split > sh.K + 1 || n_split > 65535) return SAS_ERR_INVALID_ARG;
+  if ((sh.K + n_split) / n_split > sas::kMaxDecodeBlocksPerSplit) return SAS_ERR_UNSUPPORTED;
   return from_cuda(sas::launch_decode_paged(sh, q, k_pages, v_pages, n_pages, block_table, cache_len,
                                             sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, n_split, o_part,
                                             lse_part, device_error_word(), static_cast<cudaStream_t>(stream)));

@@ -164,3 +164,12 @@ def test_gate_ablation_inputs_checked():
     assert _fwd(_p(gate_mode=4)) == INVALID
     c = _p(gate_mode=2).c()
     assert lib.sas_decode(ctypes.byref(c), A, A, A, A, None, A, None, 2, A, A, None) == INVALID  # s missing
+
+
+def test_decode_split_size_limited():
+    # a split may cover at most 64 blocks: K = 256 needs n_split >= 5
+    c = _p(top_k=256, seq_len=32768).c()
+    base = [A, A, A, A, A, A, A]
+    assert lib.sas_decode(ctypes.byref(c), *base, 1, A, A, None) == UNSUPPORTED
+    assert lib.sas_decode(ctypes.byref(c), *base, 4, A, A, None) == UNSUPPORTED
+    assert lib.sas_decode_paged(ctypes.byref(c), A, A, A, 8, A, A, A, A, A, 4, A, A, None) == UNSUPPORTED
