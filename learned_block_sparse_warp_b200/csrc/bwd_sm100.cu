@@ -126,8 +126,9 @@ struct EntryRing {
 // a ring of three slots and dO tiles in a ring of two, each with its own
 // producer warp: a Q tile lives from S = Q Kᵀ to dKᵀ += Qᵀ dZ, which spans the
 // whole step, so a third slot keeps its load off the step's critical path.
-// Four threads issue the MMAs (S, dP, dVᵀ, dKᵀ): one thread needs about 120
-// cycles per MMA issue, about twice what an N = 64 MMA takes to run. Sixteen
+// Four threads issue the MMAs (S, dP, dVᵀ, dKᵀ), so that each product's group
+// of eight dependent MMAs, about 800 cycles from first issue to completion,
+// overlaps the others instead of queueing behind them on one thread. Sixteen
 // softmax-gradient warps (four per SM sub-partition) write P as soon as S
 // allows, so dVᵀ starts before dP is consumed, then dZ.
 //

@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
     }
   } else if ((warp == 1 || warp == 3) && (warp >> 1) < n_tiles) {
     // ------------------------------------------------------------ MMA issuers, one thread per tile
-    // (a single thread needs about 70 cycles per tcgen05.mma issue)
+    // (each tile's chain S → softmax → PV is latency-bound; two threads let the
+    // two tiles' MMAs overlap)
     if (lane == 0) {
       const int r = warp >> 1;
       const uint32_t idS2 = idesc_bf16_f32(128, 128, 0, 0), idS1 = idesc_bf16_f32(128, 64, 0, 0);
