@@ -282,6 +282,14 @@ SAS_API sas_status sas_decode_noalloc(const sas_params* p, const sas_bf16* q, co
  * Diagnostics
  * ------------------------------------------------------------------------- */
 
+/* Launches one thread that waits, through the same bounded wait as the
+ * tcgen05 kernels, on an mbarrier that nothing completes. After about one
+ * second of GPU clock cycles the wait gives up and raises SAS_ERR_TIMEOUT in
+ * the device error word (read it with sas_get_device_error). It lets a caller
+ * check the timeout path and that the context stays usable afterwards; nothing
+ * faults or hangs. Asynchronous on `stream`. */
+SAS_API sas_status sas_selftest_wait_timeout(void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device. *code is SAS_OK when no kernel raised an error since the
  * last read, else the first sas_status a kernel raised (SAS_ERR_TIMEOUT or

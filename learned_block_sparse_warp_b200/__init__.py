@@ -25,7 +25,7 @@ __all__ = [
     "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd", "sas_decode",
     "sas_decode_combine", "sas_decode_paged", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string",
     "sas_version",
-    "DecodeGraph",
+    "DecodeGraph", "sas_selftest_wait_timeout",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "sas_decode_combine": [P, ctypes.c_int, vp, vp, vp, vp, vp],
         "sas_get_device_error": [vp, ctypes.POINTER(ctypes.c_int)],
         "sas_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp],
+        "sas_selftest_wait_timeout": [vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -240,6 +241,11 @@ def sas_decode_noalloc(p: Params, q, kc, vc, cache_len, s, o, lse_o=None, stream
         _ptr(vc, bf16, (B, Hkv, p.seq_len, d), "vc"), _ptr(cache_len, i32, (B,), "cache_len"),
         _ptr(s, f32, (B, Hkv, p.n_blocks), "s"), _ptr(o, bf16, (B, Hq, d), "o"), _ptr(lse_o, f32, (B, Hq), "lse_o"),
         _stream(stream)))
+
+
+def sas_selftest_wait_timeout(stream=None) -> None:
+    """One bounded wait that runs out (about a second); sas_get_device_error then reads SAS_ERR_TIMEOUT."""
+    _check("sas_selftest_wait_timeout", lib.sas_selftest_wait_timeout(_stream(stream)))
 
 
 def sas_get_device_error(stream=None) -> int:

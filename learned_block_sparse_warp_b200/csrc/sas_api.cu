@@ -30,6 +30,7 @@ cudaError_t launch_decode_paged(const Shape& sh, const uint16_t* q, const uint16
                                 int* err, cudaStream_t st);
 cudaError_t launch_decode_combine(const Shape& sh, int n_split, const float* o_part, const float* lse_part,
                                   uint16_t* o, float* lse_o, cudaStream_t st);
+cudaError_t launch_wait_timeout(int* err, cudaStream_t st);
 }  // namespace sas
 
 using sas::Shape;
@@ -238,6 +239,12 @@ sas_status sas_decode_combine(const sas_params* p, int n_split, const float* o_p
   if (n_split < 1 || n_split > sh.K + 1) return SAS_ERR_INVALID_ARG;
   return from_cuda(sas::launch_decode_combine(sh, n_split, o_part, lse_part, o, lse_o,
                                               static_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_selftest_wait_timeout(void* stream) {
+  int* err = device_error_word();
+  if (err == nullptr) return SAS_ERR_CUDA;
+  return from_cuda(sas::launch_wait_timeout(err, static_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_get_device_error(void* stream, int* code) {
