@@ -91,9 +91,11 @@ typedef struct {
   int n_q_heads;       /* Hq >= 1, a multiple of n_kv_heads */
   int n_kv_heads;      /* Hkv >= 1 */
   int head_dim;        /* d: 64 or 128 */
-  int seq_len;         /* prefill: N; decode: KV-cache capacity Lmax; a multiple of block */
+  int seq_len;         /* prefill: N; decode: KV-cache capacity Lmax; a multiple of block.
+                          SAS_ERR_UNSUPPORTED above 2^19 blocks, or when
+                          batch * n_kv_heads * blocks exceeds 2^30 */
   int block;           /* b: must be 64 */
-  int top_k;           /* K: 1..256 */
+  int top_k;           /* K: 1..2048 (K >= t selects every history block: full scope) */
   float softmax_scale; /* 0 selects 1/sqrt(d) */
   int gate_mode;       /* sas_gate_mode */
 } sas_params;

@@ -38,7 +38,7 @@ struct BwdWs {
   float* dl;       // [B, Hkv, NB, K]
   int* rev_cnt;    // [B, Hkv, NB]
   int* rev_off;    // [B, Hkv, NB + 1]
-  int* rev_list;   // [B, Hkv, NB * K]: (t << 8) | slot
+  int* rev_list;   // [B, Hkv, NB * K]: (t << kSlotBits) | slot
   float* rev_lam;  // [B, Hkv, NB * K]: log2-domain gate of each reverse-index entry
 };
 
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const int32_t* __restr
     const unsigned mask = __ballot_sync(0xffffffffu, slot >= 0);
     if (slot >= 0) {
       const int at = pos + __popc(mask & ((1u << lane) - 1u));
-      out[at] = (t << 8) | slot;
+      out[at] = (t << kSlotBits) | slot;
       if (lam != nullptr) {  // the gate of block j for query block t, log2 domain
         const size_t row = size_t(bh) * NB + t;
         lam[size_t(bh) * NB * K + at] =
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(256, 1) bwd_main_kernel(
   const int* lst = rev_list + bh * size_t(sh.NB) * sh.K + off0;
   const int n_steps = (1 + n_sel) * G;
 
-  auto step_t = [&](int e) -> int { return e == 0 ? j : (lst[e - 1] >> 8); };
+  auto step_t = [&](int e) -> int { return e == 0 ? j : (lst[e - 1] >> kSlotBits); };
   auto issue_step = [&](int st, int stage) {
     const int e = st / G, g = st % G;
     const int t = step_t(e);
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(256, 1) bwd_main_kernel(
     __syncthreads();
     const int e = st / G, g = st % G;
     const int t = step_t(e);
-    const int slot = e == 0 ? -1 : (lst[e - 1] & 255);
+    const int slot = e == 0 ? -1 : (lst[e - 1] & ((1 << kSlotBits) - 1));
     const bool diag = (e == 0);
     float lam2 = 0.f;
     if (!diag && sh.gated) {

@@ -109,15 +109,15 @@ struct EntryRing {
     }
     const int w = __shfl_sync(0xffffffffu, w_cur, e & 31);
     lam2 = __shfl_sync(0xffffffffu, l_cur, e & 31);
-    t = e == 0 ? j : (w >> 8);
-    slot = e == 0 ? -1 : (w & 255);
+    t = e == 0 ? j : (w >> kSlotBits);
+    slot = e == 0 ? -1 : (w & ((1 << kSlotBits) - 1));
     if (e == 0) lam2 = 0.f;
   }
   // t of entry e of the next batch at most, for prefetching (no state change)
   __device__ int peek_t(int e, int j) const {
     const int src = (e >> 5) == batch ? w_cur : w_nxt;
     const int w = __shfl_sync(0xffffffffu, src, e & 31);
-    return e == 0 ? j : (w >> 8);
+    return e == 0 ? j : (w >> kSlotBits);
   }
 };
 

@@ -12,7 +12,8 @@
 namespace sas {
 
 constexpr int kBlock = 64;          // tokens per block (b)
-constexpr int kMaxTopK = 256;       // largest K the kernels accept
+constexpr int kMaxTopK = 2048;      // largest K the kernels accept
+constexpr int kSlotBits = 12;       // reverse-index entry: (t << kSlotBits) | slot, slot < K <= 4096
 constexpr int kMaxDecodeBlocksPerSplit = 64;  // ceil((K + 1) / n_split) fits the decode task list
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;

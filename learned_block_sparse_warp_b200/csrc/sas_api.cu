@@ -81,13 +81,16 @@ sas_status make_shape(const sas_params* p, Shape* sh) {
   if (p->gate_mode < SAS_GATE_LOG_SOFTMAX || p->gate_mode > SAS_GATE_LOGIT) return SAS_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.f) || isinf(p->softmax_scale)) return SAS_ERR_INVALID_ARG;
   if (p->top_k > sas::kMaxTopK) return SAS_ERR_INVALID_ARG;
+  static_assert(sas::kMaxTopK <= (1 << sas::kSlotBits), "reverse-index slot field");
   if (p->block != sas::kBlock) return SAS_ERR_UNSUPPORTED;
   if (p->head_dim != 64 && p->head_dim != 128) return SAS_ERR_UNSUPPORTED;
   if (p->seq_len % sas::kBlock != 0) return SAS_ERR_INVALID_ARG;
   if (p->batch > 65535 || p->n_q_heads > 65535) return SAS_ERR_UNSUPPORTED;
-  // keep every flattened row index of the scores within int range
+  // keep every flattened row index of the scores within int range, and every
+  // reverse-index entry (t << kSlotBits) | slot positive
   const long long nb = p->seq_len / sas::kBlock;
-  if ((long long)p->batch * p->n_kv_heads * nb > (1LL << 30) || nb > (1 << 23)) return SAS_ERR_UNSUPPORTED;
+  if ((long long)p->batch * p->n_kv_heads * nb > (1LL << 30) || nb > (1LL << (31 - sas::kSlotBits)))
+    return SAS_ERR_UNSUPPORTED;
   sh->B = p->batch;
   sh->Hq = p->n_q_heads;
   sh->Hkv = p->n_kv_heads;

@@ -65,7 +65,8 @@ def _fwd(p, q=A, k=A, v=A, s=A, idx=A, lse_s=A, o=A, lse_o=None):
     (dict(seq_len=0), INVALID),
     (dict(n_q_heads=3), INVALID),
     (dict(top_k=0), INVALID),
-    (dict(top_k=257), INVALID),
+    (dict(top_k=2049), INVALID),
+    (dict(seq_len=64 * (2 ** 19 + 1), n_q_heads=1, n_kv_heads=1), UNSUPPORTED),
     (dict(batch=0), INVALID),
     (dict(gate_mode=7), INVALID),
     (dict(softmax_scale=-1.0), INVALID),
