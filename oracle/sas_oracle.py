@@ -22,6 +22,9 @@ pages it cites:
   softmax-normalised gate log g_m = s_m − LSE(s), the gate gradient with the gate
   inside the softmax, dg_m = Σ_i (p̃_i/g_m) dOᵀ(v_i − o), and "sparse scope"
   training.
+* [PBS]: the gist.science page "Sparser Block-Sparse Attention via Token
+  Permutation". Section 4 (実装) estimates block importance from mean-pooled
+  keys.
 
 Readings where the pages are silent or garbled (page 1's display equations
 were lost when the page was extracted):
@@ -46,6 +49,13 @@ were lost when the page was extracted):
    maps logical blocks to pages. Paging changes where tokens are stored, not
    what the step computes: ``decode_paged`` is ``decode`` on the gathered
    dense cache.
+9. Selector scoring for decode. The pages' selector is a trained network
+   whose weights are not available. The stand-in scores history block m by
+   the mean-pooled key: s_m = scale · ⟨q̄, k̄_m⟩, where k̄_m is the mean of the
+   block's keys and q̄ the mean of the new token's queries over the KV head's
+   group. This is the learned selector with identity projections. It also
+   equals the mean over the block's tokens and the group's heads of the
+   token-level logits.
 
 All arithmetic is float64. Inputs are taken as given; the generators round
 them to bf16 before either side sees them.
@@ -479,3 +489,49 @@ def decode_combine(o_part: np.ndarray, lse_part: np.ndarray):
         w = np.exp(lse_part[ix] - tot)
         o[ix] = w @ o_part[ix]
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Selector scoring for decode from mean-pooled keys (reading 9).
+# [SAS-summary] §전제와 한계: the decode step's selector scoring and Top-K
+# ranking grow with the context, unlike the attention itself. [PBS] §4 実装:
+# block importance is estimated from mean-pooled keys.
+# ---------------------------------------------------------------------------
+def block_mean_keys(k, block: int = 64) -> np.ndarray:
+    """k [B, Hkv, L, d] -> k̄ [B, Hkv, L // block, d], the mean of each block's keys."""
+    k = np.asarray(k, np.float64)
+    B, H, L, d = k.shape
+    nb = L // block
+    out = np.zeros((B, H, nb, d))
+    for m in range(nb):
+        out[:, :, m] = k[:, :, m * block:(m + 1) * block].sum(axis=2) / block
+    return out
+
+
+def decode_scores(q, kmean, cache_len, block: int = 64, softmax_scale: Optional[float] = None) -> np.ndarray:
+    """Selector scores of a decode step: s [B, Hkv, NKB].
+
+    s[b, h, m] = scale · ⟨q̄, k̄_m⟩ for the history blocks m < c of sequence b,
+    with q̄ the mean of the new token's query vectors over the KV head's group.
+    Entries m ≥ c are NaN: nothing reads them.
+    """
+    q = np.asarray(q, np.float64)
+    kmean = np.asarray(kmean, np.float64)
+    B, Hq, d = q.shape
+    Hkv, NKB = kmean.shape[1], kmean.shape[2]
+    G = Hq // Hkv
+    scale = _scale(d, softmax_scale)
+    s = np.full((B, Hkv, NKB), np.nan)
+    for b in range(B):
+        c = (int(cache_len[b]) - 1) // block
+        for h in range(Hkv):
+            qbar = q[b, h * G:(h + 1) * G].mean(axis=0)
+            s[b, h, :c] = scale * (kmean[b, h, :c] @ qbar)
+    return s
+
+
+def decode_select_scored(q, kmean, cache_len, K: int, block: int = 64, softmax_scale: Optional[float] = None):
+    """Scores from block-mean keys, then the decode-form Top-K and LSE(s): (s, idx, lse_s)."""
+    s = decode_scores(q, kmean, cache_len, block, softmax_scale)
+    idx, lse = decode_select(s, cache_len, K, block)
+    return s, idx, lse

@@ -6,7 +6,9 @@ None of these checks runs the oracle against a copy of itself. They use:
 * torch's scaled_dot_product_attention in fp64 (the dense special cases),
 * central finite differences (every gradient, including ds),
 * the pages' own gate-gradient formula evaluated token by token,
-* the invariances the pages state (shift of s, permutation inside a block).
+* the invariances the pages state (shift of s, permutation inside a block),
+* for the block-mean selector scores: running token sums, and the mean of the
+  token-level logits over a block and a head group.
 """
 import json
 import math
@@ -487,3 +489,68 @@ def test_gate_ablations_have_their_closed_forms():
         a = O.log_gate(s_hist[1:4], [0, 2], mode)
         b = O.log_gate(s_hist[1:4] + 1.5, [0, 2], mode)
         assert (np.abs(a - b).max() < 1e-12) == inv
+
+
+# ---------------------------------------------------------------------------
+# Selector scoring from block-mean keys (decode)
+# ---------------------------------------------------------------------------
+def test_block_mean_keys_by_prefix_sums():
+    """Each block mean is a difference of running token sums over 64."""
+    g = np.random.default_rng(31)
+    k = g.standard_normal((2, 3, 64 * 5 + 17, 8))
+    km = O.block_mean_keys(k)
+    assert km.shape == (2, 3, 5, 8)
+    csum = np.concatenate([np.zeros((2, 3, 1, 8)), np.cumsum(k, axis=2)], axis=2)
+    for m in range(5):
+        np.testing.assert_allclose(km[:, :, m] * 64, csum[:, :, 64 * (m + 1)] - csum[:, :, 64 * m], rtol=0, atol=1e-11)
+
+
+def test_block_mean_of_a_constant_block_is_that_key():
+    g = np.random.default_rng(32)
+    u = np.round(g.standard_normal((4, 16)) * 64) / 64  # short mantissas: every partial sum is exact
+    k = np.repeat(u, 64, axis=0)[None, None]  # block m holds 64 copies of u[m]
+    assert np.array_equal(O.block_mean_keys(k)[0, 0], u)
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_decode_scores_are_mean_token_logits(G):
+    """s_m equals the mean over the block's tokens and the group's heads of scale·q_g·k_j."""
+    g = np.random.default_rng(33 + G)
+    B, Hkv, d, L = 2, 2, 16, 64 * 6
+    q = g.standard_normal((B, Hkv * G, d))
+    k = g.standard_normal((B, Hkv, L, d))
+    cache_len = np.array([L, 64 * 3 + 5])
+    s = O.decode_scores(q, O.block_mean_keys(k), cache_len)
+    scale = 1 / math.sqrt(d)
+    for b in range(B):
+        c = (int(cache_len[b]) - 1) // 64
+        for h in range(Hkv):
+            logits = scale * (q[b, h * G:(h + 1) * G] @ k[b, h].T)  # [G, L]
+            want = logits[:, :64 * c].reshape(G, c, 64).mean(axis=(0, 2))
+            np.testing.assert_allclose(s[b, h, :c], want, rtol=1e-12, atol=1e-12)
+            assert np.isnan(s[b, h, c:]).all()
+
+
+def test_scored_selection_ranks_aligned_blocks_first():
+    """A block whose keys all point along the query ranks first; one pointing against it, last."""
+    g = np.random.default_rng(35)
+    d, G, L = 32, 4, 64 * 40 + 1
+    u = g.standard_normal(d)
+    u /= np.linalg.norm(u)
+    q = g.standard_normal((1, G, d)) + 4 * u
+    k = g.standard_normal((1, 1, L, d))
+    k[0, 0, 64 * 7:64 * 8] += 4 * u
+    k[0, 0, 64 * 22:64 * 23] -= 4 * u
+    s, idx, lse = O.decode_select_scored(q, O.block_mean_keys(k), np.array([L]), K=39)
+    row = s[0, 0, :40]
+    assert int(np.argmax(row)) == 7 and int(np.argmin(row)) == 22
+    # K = 39 of 40 history blocks: every block but the anti-aligned one, ascending
+    assert idx[0, 0].tolist() == [m for m in range(40) if m != 22]
+    assert lse[0, 0] == pytest.approx(math.log(np.exp(row).sum()), rel=1e-12)
+
+
+def test_scored_selection_without_history():
+    q = np.ones((2, 4, 8))
+    k = np.ones((2, 2, 128, 8))
+    s, idx, lse = O.decode_select_scored(q, O.block_mean_keys(k), np.array([1, 64]), K=3)
+    assert (idx == -1).all() and np.isneginf(lse).all() and np.isnan(s).all()
