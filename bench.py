@@ -448,11 +448,120 @@ def run_gpu(args, rank, world, local_rank):
         if sas.sas_get_device_error(stream) != 0:
             raise RuntimeError("device error during decode")
 
+    # ---------------- long-context decode that scores its own history ----------------
+    if args.only in ("all", "long_decode") and not args.no_decode:
+        try:
+            line["long_decode"] = long_decode_section(args, sas, stream, dev, pk, dist, world)
+        except Exception as e:  # a supplementary section: its failure is reported, not the whole line lost
+            if args.only == "long_decode":
+                raise
+            line["long_decode"] = {"error": f"{type(e).__name__}: {e}"[:400]}
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only in ("all", "train"):
         line["cpu_baseline"] = oracle_baseline(W.WORKLOADS[TRAIN], budget_s=args.cpu_budget)
     if dist is not None:
         dist.destroy_process_group()
     return line
+
+
+# ---------------------------------------------------------------------------
+# long-context decode: block-mean update, fused scoring + Top-K, split-K, merge
+# ---------------------------------------------------------------------------
+LONG_DECODE = [  # (batch, cache tokens): the context lengths and batch sizes of the pages' decode measurements
+    (1, 65536), (1, 262144), (1, 524288), (8, 65536)]
+
+
+def long_decode_section(args, sas, stream, dev, pk, dist, world):
+    import torch
+    out_rows = []
+    Hq, Hkv, d, K = 32, 8, 128, 16
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            fn()
+        return g
+
+    def timed(g):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        g.replay()
+        ev[1].record(stream)
+        return ev
+
+    for B, L in LONG_DECODE:
+        NB = L // 64
+        p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=L, top_k=K,
+                       gate_mode=sas.SAS_GATE_NONE)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1000 + B * 7 + NB)
+        with torch.cuda.stream(stream):
+            kc = torch.randn((B, Hkv, L, d), generator=gen, device=dev, dtype=torch.bfloat16)
+            vc = torch.randn((B, Hkv, L, d), generator=gen, device=dev, dtype=torch.bfloat16)
+            q = torch.randn((B, Hq, d), generator=gen, device=dev, dtype=torch.bfloat16)
+            cl = torch.full((B,), L, dtype=torch.int32, device=dev)
+            km = torch.empty((B, Hkv, NB, d), dtype=torch.bfloat16, device=dev)
+            sas.sas_block_mean_keys(p, kc, km, stream=stream)  # after the prefill: every block
+            s = torch.empty((B, Hkv, NB), dtype=torch.float32, device=dev)
+        n_split = K + 1
+        od = sas.empty_decode_outputs(p, n_split, device=dev)
+        step = sas.DecodeGraph(p, q, kc, vc, cl, s, n_split, od, stream=stream, kmean=km)
+        g_mean = capture(lambda: sas.sas_block_mean_keys(p, kc, km, cache_len=cl))
+        g_sel = capture(lambda: sas.sas_decode_select_scored(p, q, km, cl, s, od["idx"], od["lse_s"]))
+        g_split = capture(lambda: sas.sas_decode(p, q, kc, vc, cl, s, od["idx"], od["lse_s"], n_split, od["o_part"],
+                                                 od["lse_part"]))
+        g_comb = capture(lambda: sas.sas_decode_combine(p, n_split, od["o_part"], od["lse_part"], od["o"],
+                                                        od["lse_o"]))
+        # unfused comparison: the scores by a library batched matmul, then the separate Top-K kernel
+        qbar = torch.empty((B * Hkv, d, 1), dtype=torch.bfloat16, device=dev)
+        s_mm = torch.empty((B * Hkv, NB, 1), dtype=torch.bfloat16, device=dev)
+        s_un = torch.empty((B, Hkv, NB), dtype=torch.float32, device=dev)
+
+        def unfused():
+            qbar.copy_(q.view(B * Hkv, Hq // Hkv, d).float().mean(dim=1).mul_(d ** -0.5).unsqueeze(-1))
+            torch.bmm(km.view(B * Hkv, NB, d), qbar, out=s_mm)
+            s_un.view(B * Hkv, NB).copy_(s_mm.view(B * Hkv, NB))
+            sas.sas_topk_select(p, s_un, od["idx"], od["lse_s"], cache_len=cl)
+
+        with torch.cuda.stream(stream):
+            unfused()  # first call outside capture: the library GEMM's handle is created here
+        g_unf = capture(unfused)
+        graphs = {"step": step.graph, "mean_update": g_mean, "select": g_sel, "split": g_split, "combine": g_comb,
+                  "select_unfused": g_unf}
+        times = {k: [] for k in graphs}
+        with torch.cuda.stream(stream):
+            for _ in range(max(3, args.warmup)):
+                for g in graphs.values():
+                    g.replay()
+            for _ in range(max(10, args.steps)):
+                for key, g in graphs.items():
+                    torch.sum(flush, dim=0, out=flush_sink)
+                    times[key].append(timed(g))
+        torch.cuda.synchronize()
+        med = {k: statistics.median(e[0].elapsed_time(e[1]) for e in evs) for k, evs in times.items()}
+        if sas.sas_get_device_error(stream) != 0:
+            raise RuntimeError("device error during long-context decode")
+        step_ms = max_over_ranks(dist, med["step"], dev)
+        c = (L - 1) // 64
+        sel_bytes = B * Hkv * c * (d * 2 + 4) + B * Hq * d * 2 + B * Hkv * (K + 1) * 4
+        gbs = sel_bytes / (med["select"] * 1e-3) / 1e9
+        out_rows.append({
+            "batch": B, "cache_len": L, "top_k": K, "heads": f"{Hq}/{Hkv}", "head_dim": d,
+            "ms_per_step": step_ms, "tok_per_s": job_rate(B, world, step_ms * 1e-3),
+            "breakdown_ms": {k: med[k] for k in ("mean_update", "select", "split", "combine")},
+            "select_share": med["select"] / (med["mean_update"] + med["select"] + med["split"] + med["combine"]),
+            "select_unfused_ms": med["select_unfused"],
+            "select_roofline": {"bound": "hbm", "kernel": "select_scored_kernel (sas_decode_select_scored)",
+                                "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
+                                "algorithmic_bytes": sel_bytes}})
+        del step, g_mean, g_sel, g_split, g_comb, g_unf, graphs, kc, vc, km, s, od
+        torch.cuda.empty_cache()
+    return {"workloads": out_rows, "gate": "none (inference form)", "n_split": K + 1,
+            "data": "synthetic: q, k, v ~ N(0, 1) bf16 from a seeded device generator",
+            "launch": "one CUDA graph per step: block-mean update, fused scoring + Top-K, split-K, merge (PDL-chained)",
+            "l2": "flushed (252 MB read) before every timed replay", "gpu_launches_per_step": 4}
 
 
 # ---------------------------------------------------------------------------
@@ -489,7 +598,7 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sas", "reference"], default="sas")
-    ap.add_argument("--only", choices=["all", "train", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "train", "decode", "long_decode"], default="all",
                     help="run only one workload (for profiling); the JSON line needs 'all'")
     ap.add_argument("--n-split", type=int, default=0, help="decode splits (0: K + 1)")
     ap.add_argument("--no-e2e", action="store_true")

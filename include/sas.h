@@ -237,6 +237,51 @@ SAS_API sas_status sas_decode_combine(const sas_params* p, int n_split, const fl
                               sas_bf16* o, float* lse_o, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Selector scoring fused with Top-K for long decode caches (SAS summary
+ * §전제와 한계: in decode, the selector's scoring and the Top-K ranking grow
+ * with the context while the attention does not. PBS §4: block importance
+ * from mean-pooled keys.)
+ * ------------------------------------------------------------------------- */
+
+/* Block-mean keys: kmean[b, h, m, :] = (1/64) Σ_{j<64} k[b, h, 64m + j, :],
+ * summed in fp32 and rounded once to bf16.
+ *   k          bf16 [B, Hkv, Lmax, d] (Lmax = seq_len), the K cache.
+ *   cache_len  NULL: every block m < Lmax/64 of every sequence is written.
+ *              int32 [B]: the decode update. For each sequence whose
+ *              cache_len[b] is a multiple of 64, only block cache_len[b]/64 − 1
+ *              (the block the newest token completed) is written; nothing is
+ *              written for the other sequences. A cache_len outside
+ *              [1, Lmax] raises SAS_ERR_DEVICE_INDEX.
+ *   kmean      bf16 [B, Hkv, Lmax/64, d]. Output, caller-owned.
+ * Blocks must be complete when summarised: a block with tokens past the
+ * sequence's cache_len is summarised over whatever the cache holds there. */
+SAS_API sas_status sas_block_mean_keys(const sas_params* p, const sas_bf16* k, const int32_t* cache_len,
+                                       sas_bf16* kmean, void* stream);
+
+/* Selector scores of one decode step and their Top-K, in one launch.
+ *   s[b, h, m] = scale · ⟨q̄, kmean[b, h, m]⟩ for the history blocks m < c,
+ *   c = (cache_len[b] − 1)/64, with q̄ = (1/G) Σ_g q[b, h·G + g] and scale
+ *   p->softmax_scale (0 selects 1/sqrt(d)). Then, as the decode form of
+ *   sas_topk_select on these scores: idx = the n = min(K, c) highest-scoring
+ *   history blocks, ties to the lower m, ascending, padded with −1; lse_s =
+ *   log Σ_{m<c} exp s[b, h, m], −inf when c = 0.
+ *   q          bf16 [B, Hq, d]
+ *   kmean      bf16 [B, Hkv, NKB, d] from sas_block_mean_keys
+ *   cache_len  int32 [B], 1 <= L <= seq_len (otherwise SAS_ERR_DEVICE_INDEX,
+ *              and the row is treated as having no history)
+ *   s          fp32 [B, Hkv, NKB]. Output: entries m < c are written, the
+ *              rest are left as they were. sas_decode reads it for the gate.
+ *   idx        int32 [B, Hkv, K]. Output.
+ *   lse_s      fp32 [B, Hkv]. Output, may be NULL.
+ * The selection is exact for the scores written to s (a full sort of s would
+ * pick the same blocks). Each row is split over a cluster of up to 8 CTAs,
+ * each holding at most 53,248 scores in shared memory: SAS_ERR_UNSUPPORTED
+ * beyond 8 × 53,248 history blocks (about 27M tokens). */
+SAS_API sas_status sas_decode_select_scored(const sas_params* p, const sas_bf16* q, const sas_bf16* kmean,
+                                            const int32_t* cache_len, float* s, int32_t* idx, float* lse_s,
+                                            void* stream);
+
+/* ---------------------------------------------------------------------------
  * Decode step that allocates nothing. The paper has no counterpart to this
  * entry point; it exists for callers of this library that cannot allocate.
  * ------------------------------------------------------------------------- */

@@ -25,7 +25,8 @@ __all__ = [
     "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd", "sas_decode",
     "sas_decode_combine", "sas_decode_paged", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string",
     "sas_version",
-    "DecodeGraph", "sas_selftest_wait_timeout",
+    "DecodeGraph", "sas_selftest_wait_timeout", "sas_block_mean_keys", "sas_decode_select_scored",
+    "decode_step_scored",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
@@ -71,6 +72,8 @@ def _load() -> ctypes.CDLL:
         "sas_get_device_error": [vp, ctypes.POINTER(ctypes.c_int)],
         "sas_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp],
         "sas_selftest_wait_timeout": [vp],
+        "sas_block_mean_keys": [P, vp, vp, vp, vp],
+        "sas_decode_select_scored": [P, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -243,6 +246,24 @@ def sas_decode_noalloc(p: Params, q, kc, vc, cache_len, s, o, lse_o=None, stream
         _stream(stream)))
 
 
+def sas_block_mean_keys(p: Params, k, kmean, cache_len=None, stream=None) -> None:
+    """k̄[b, h, m] = mean of block m's 64 keys (bf16). With cache_len, only each sequence's just-completed block."""
+    B, Hkv, d = p.batch, p.n_kv_heads, p.head_dim
+    _check("sas_block_mean_keys", lib.sas_block_mean_keys(
+        ctypes.byref(p.c()), _ptr(k, bf16, (B, Hkv, p.seq_len, d), "k"), _ptr(cache_len, i32, (B,), "cache_len"),
+        _ptr(kmean, bf16, (B, Hkv, p.n_blocks, d), "kmean"), _stream(stream)))
+
+
+def sas_decode_select_scored(p: Params, q, kmean, cache_len, s, idx, lse_s=None, stream=None) -> None:
+    """Selector scores from block-mean keys (written to s for m < c) and their decode-form Top-K, fused."""
+    B, Hq, Hkv, d = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim
+    sh = _shapes(p, True)
+    _check("sas_decode_select_scored", lib.sas_decode_select_scored(
+        ctypes.byref(p.c()), _ptr(q, bf16, (B, Hq, d), "q"), _ptr(kmean, bf16, (B, Hkv, p.n_blocks, d), "kmean"),
+        _ptr(cache_len, i32, (B,), "cache_len"), _ptr(s, f32, sh["s"], "s"), _ptr(idx, i32, sh["idx"], "idx"),
+        _ptr(lse_s, f32, sh["lse_s"], "lse_s"), _stream(stream)))
+
+
 def sas_selftest_wait_timeout(stream=None) -> None:
     """One bounded wait that runs out (about a second); sas_get_device_error then reads SAS_ERR_TIMEOUT."""
     _check("sas_selftest_wait_timeout", lib.sas_selftest_wait_timeout(_stream(stream)))
@@ -314,6 +335,16 @@ def decode_step(p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, str
     sas_decode_combine(p, n_split, out["o_part"], out["lse_part"], out["o"], out["lse_o"], stream=stream)
 
 
+def decode_step_scored(p: Params, q, kc, vc, kmean, cache_len, s, n_split: int, out: dict, stream=None) -> None:
+    """A decode step that scores its own history: update the block means of any block the newest token
+    completed, score and select in one launch (s is written), split-K attention, merge."""
+    sas_block_mean_keys(p, kc, kmean, cache_len=cache_len, stream=stream)
+    sas_decode_select_scored(p, q, kmean, cache_len, s, out["idx"], out["lse_s"], stream=stream)
+    sas_decode(p, q, kc, vc, cache_len, s, out["idx"], out["lse_s"], n_split, out["o_part"], out["lse_part"],
+               stream=stream)
+    sas_decode_combine(p, n_split, out["o_part"], out["lse_part"], out["o"], out["lse_o"], stream=stream)
+
+
 class DecodeGraph:
     """A decode step (select, split-K, merge) captured once as a CUDA graph.
 
@@ -324,16 +355,20 @@ class DecodeGraph:
     launch, so each one's launch overlaps the tail of the one before.
     """
 
-    def __init__(self, p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, stream=None):
-        self.args = (p, q, kc, vc, cache_len, s, n_split, out)
+    def __init__(self, p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, stream=None, kmean=None):
+        # with kmean, the step scores its own history (decode_step_scored) and s is an output
+        if kmean is None:
+            self.step, self.args = decode_step, (p, q, kc, vc, cache_len, s, n_split, out)
+        else:
+            self.step, self.args = decode_step_scored, (p, q, kc, vc, kmean, cache_len, s, n_split, out)
         side = torch.cuda.Stream() if stream is None else stream
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):  # first call outside capture: kernel attributes get set here
-            decode_step(*self.args, stream=side)
+            self.step(*self.args, stream=side)
         torch.cuda.current_stream().wait_stream(side)
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph, stream=side, capture_error_mode="thread_local"):
-            decode_step(*self.args, stream=side)
+            self.step(*self.args, stream=side)
 
     def replay(self) -> None:
         self.graph.replay()

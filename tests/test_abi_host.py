@@ -174,3 +174,31 @@ def test_decode_split_size_limited():
     assert lib.sas_decode(ctypes.byref(c), *base, 1, A, A, None) == UNSUPPORTED
     assert lib.sas_decode(ctypes.byref(c), *base, 4, A, A, None) == UNSUPPORTED
     assert lib.sas_decode_paged(ctypes.byref(c), A, A, A, 8, A, A, A, A, A, 4, A, A, None) == UNSUPPORTED
+
+
+def test_block_mean_keys_checked():
+    c = _p().c()
+    f = lib.sas_block_mean_keys
+    assert f(None, A, None, A, None) == INVALID
+    assert f(ctypes.byref(c), None, None, A, None) == INVALID
+    assert f(ctypes.byref(c), A, None, None, None) == INVALID
+    assert f(ctypes.byref(c), A + 2, None, A, None) == INVALID
+    assert f(ctypes.byref(c), A, A + 4, A, None) == INVALID  # cache_len misaligned
+    assert f(ctypes.byref(_p(head_dim=96).c()), A, None, A, None) == UNSUPPORTED
+
+
+def test_decode_select_scored_checked():
+    c = _p().c()
+
+    def call(params=c, q=A, kmean=A, cl=A, s=A, idx=A, lse=None):
+        return lib.sas_decode_select_scored(ctypes.byref(params) if params is not None else None, q, kmean, cl, s,
+                                            idx, lse, None)
+
+    assert call(params=None) == INVALID
+    for kw in ("q", "kmean", "cl", "s", "idx"):
+        assert call(**{kw: None}) == INVALID, kw
+    assert call(lse=A + 4) == INVALID
+    assert call(params=_p(head_dim=96).c()) == UNSUPPORTED
+    # a row of more than 8 x 53,248 history blocks does not fit a cluster's shared memory
+    big = _p(n_q_heads=1, n_kv_heads=1, seq_len=64 * (8 * 53248 + 2)).c()
+    assert call(params=big) == UNSUPPORTED
