@@ -56,6 +56,13 @@ were lost when the page was extracted):
    group. This is the learned selector with identity projections. It also
    equals the mean over the block's tokens and the group's heads of the
    token-level logits.
+10. The gate outside the softmax. [SAS-summary] §무엇과 다른가 contrasts it with
+    the gate inside: outside, the attention probabilities are those of the
+    plain logits and the gate only re-weights the values, with dg_m = Σ p_i dOᵀv_i
+    over block m's tokens. Read with the method's g = softmax(s) and g0 = 1: p is
+    the softmax over the plain logits of the whole attended set, and the output
+    o = Σ_i g_{m(i)} p_i v_i is not renormalised. dl = g·dg feeds the same chain
+    to ds as the gate inside.
 
 All arithmetic is float64. Inputs are taken as given; the generators round
 them to bf16 before either side sees them.
@@ -74,6 +81,10 @@ GATE_NONE = 1  # inference form (Algorithm 2): Top-K only, no gate
 # to 0. Both stay inside the softmax in log form.
 GATE_LOG_SIGMOID = 2  # log g_m = log σ(s_m)
 GATE_LOGIT = 3  # log g_m = s_m
+# The gate outside the softmax ([SAS-summary] §무엇과 다른가, the first design
+# choice): g = softmax(s) multiplies the values of its block after a softmax
+# over the plain logits, o = Σ_i g_{m(i)} p_i v_i.
+GATE_SOFTMAX_OUTSIDE = 4
 
 
 def _scale(d: int, softmax_scale: Optional[float]) -> float:
@@ -163,6 +174,7 @@ def log_gate(s_hist: np.ndarray, selected: Sequence[int], gate_mode: int) -> np.
         return np.array([_log_sigmoid(float(s_hist[m])) for m in selected], dtype=np.float64)
     if gate_mode == GATE_LOGIT:
         return np.array([float(s_hist[m]) for m in selected], dtype=np.float64)
+    # the softmax-normalised gate, inside (log g in the logits) or outside (g on the values)
     lse = logsumexp(s_hist)
     return np.array([float(s_hist[m]) - lse for m in selected], dtype=np.float64)
 
@@ -176,7 +188,7 @@ def gate_score_gradient(s_hist: np.ndarray, selected: Sequence[int], dl_sel: np.
     """
     sh = np.asarray(s_hist, np.float64)
     ds_row = np.zeros(len(sh))
-    if gate_mode == GATE_LOG_SOFTMAX:
+    if gate_mode in (GATE_LOG_SOFTMAX, GATE_SOFTMAX_OUTSIDE):
         ds_row = -np.exp(sh - logsumexp(sh)) * float(np.sum(dl_sel))
     for m, x in zip(selected, dl_sel):
         if gate_mode == GATE_LOG_SIGMOID:
@@ -195,6 +207,14 @@ def _gathered_tokens(t: int, selected: Sequence[int], block: int, n_cur: int) ->
 # ---------------------------------------------------------------------------
 # Forward: Eq. (9) of [SAS-explainer] §仕組み, o = softmax(qK_Sᵀ + log g_S) V_S
 # ---------------------------------------------------------------------------
+def _gate_placement(lam_tok: np.ndarray, gate_mode: int):
+    """(logit bias, value weight) per gathered token: (log g, 1) for a gate inside the
+    softmax, (0, g) for the gate outside it. The current block has log g = 0 either way."""
+    if gate_mode == GATE_SOFTMAX_OUTSIDE:
+        return np.zeros_like(lam_tok), np.exp(lam_tok)
+    return lam_tok, np.ones_like(lam_tok)
+
+
 def _block_logits(qb, Kst, lam_tok, scale, causal_n):
     """z = scale·q Kᵀ + log g, with the causal mask inside the current block.
 
@@ -237,16 +257,17 @@ def forward(q, k, v, s, idx, block: int = 64, gate_mode: int = GATE_LOG_SOFTMAX,
                 lam = log_gate(s[b, h, t, :t], sel, gate_mode)
                 tok = _gathered_tokens(t, sel, block, block)
                 lam_tok = np.concatenate([np.zeros(block), np.repeat(lam, block)])
+                z_bias, g_tok = _gate_placement(lam_tok, gate_mode)
                 Kst, Vst = k[b, h, tok], v[b, h, tok]
                 rows = slice(block * t, block * t + block)
                 for g in range(G):
                     hq = h * G + g
-                    z = _block_logits(q[b, hq, rows], Kst, lam_tok, scale, block)
+                    z = _block_logits(q[b, hq, rows], Kst, z_bias, scale, block)
                     zmax = z.max(axis=1, keepdims=True)
                     e = np.exp(z - zmax)
                     den = e.sum(axis=1, keepdims=True)
                     P = e / den
-                    o[b, hq, rows] = P @ Vst
+                    o[b, hq, rows] = (P * g_tok) @ Vst
                     L[b, hq, rows] = (zmax + np.log(den))[:, 0]
     return o, L
 
@@ -293,25 +314,29 @@ def backward(q, k, v, s, idx, do, block: int = 64, gate_mode: int = GATE_LOG_SOF
                 lam = log_gate(s[b, h, t, :t], sel, gate_mode)
                 tok = _gathered_tokens(t, sel, block, block)
                 lam_tok = np.concatenate([np.zeros(block), np.repeat(lam, block)])
+                z_bias, g_tok = _gate_placement(lam_tok, gate_mode)
                 Kst, Vst = k[b, h, tok], v[b, h, tok]
                 rows = slice(block * t, block * t + block)
                 dlam_tok = np.zeros(len(tok))
                 for g in range(G):
                     hq = h * G + g
-                    z = _block_logits(q[b, hq, rows], Kst, lam_tok, scale, block)
+                    z = _block_logits(q[b, hq, rows], Kst, z_bias, scale, block)
                     zmax = z.max(axis=1, keepdims=True)
                     e = np.exp(z - zmax)
                     P = e / e.sum(axis=1, keepdims=True)
-                    ob = P @ Vst if o is None else np.asarray(o[b, hq, rows], np.float64)
+                    ob = (P * g_tok) @ Vst if o is None else np.asarray(o[b, hq, rows], np.float64)
                     dOb = do[b, hq, rows]
-                    dP = dOb @ Vst.T  # ∂⟨dO,o⟩/∂P
-                    Drow = np.sum(dOb * ob, axis=1, keepdims=True)  # = Σ_j P_ij dP_ij
-                    dZ = P * (dP - Drow)  # ∂/∂z through the row softmax
+                    dP = dOb @ Vst.T  # ∂⟨dO,o⟩/∂(the weight of v_j): g_j p_j is that weight
+                    Drow = np.sum(dOb * ob, axis=1, keepdims=True)  # = Σ_j P_ij g_j dP_ij
+                    dZ = P * (g_tok * dP - Drow)  # ∂/∂z through the row softmax
                     dq[b, hq, rows] += scale * (dZ @ Kst)
                     # tok holds distinct positions, so fancy-index += sums each row once
                     dk[b, h, tok] += scale * (dZ.T @ q[b, hq, rows])
-                    dv[b, h, tok] += P.T @ dOb
-                    dlam_tok += dZ.sum(axis=0)
+                    dv[b, h, tok] += (P * g_tok).T @ dOb
+                    if gate_mode == GATE_SOFTMAX_OUTSIDE:
+                        dlam_tok += (P * g_tok * dP).sum(axis=0)  # g ∂/∂g: ∂g/∂log g = g
+                    else:
+                        dlam_tok += dZ.sum(axis=0)
                 if gate_mode == GATE_NONE or t == 0:
                     continue
                 dl_sel = dlam_tok[block:].reshape(len(sel), block).sum(axis=1)
@@ -400,9 +425,10 @@ def _decode_partial(qv, kc, vc, blocks, L, s_hist, sel, gate_mode, scale, block)
             toks.append(np.arange(block * m, block * m + block))
             lt.append(np.full(block, lam[m]))
     toks = np.concatenate(toks)
-    z = scale * (kc[toks] @ qv) + np.concatenate(lt)
+    z_bias, g_tok = _gate_placement(np.concatenate(lt), gate_mode)
+    z = scale * (kc[toks] @ qv) + z_bias
     lse = logsumexp(z)
-    return np.exp(z - lse) @ vc[toks], lse
+    return (np.exp(z - lse) * g_tok) @ vc[toks], lse
 
 
 def decode(q, kc, vc, cache_len, s, K: int, block: int = 64, gate_mode: int = GATE_NONE,

@@ -289,7 +289,8 @@ def test_gate_reweights_probabilities():
 # ---------------------------------------------------------------------------
 # Gradients: central finite differences and the pages' gate-gradient formula
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("gate_mode", [O.GATE_LOG_SOFTMAX, O.GATE_NONE, O.GATE_LOG_SIGMOID, O.GATE_LOGIT])
+@pytest.mark.parametrize("gate_mode", [O.GATE_LOG_SOFTMAX, O.GATE_NONE, O.GATE_LOG_SIGMOID, O.GATE_LOGIT,
+                                       O.GATE_SOFTMAX_OUTSIDE])
 def test_gradients_finite_differences(gate_mode):
     blk, N, d, K = 4, 16, 4, 2
     q, k, v, do, s = _rand_case(B=1, Hq=2, Hkv=1, N=N, d=d, block=blk, seed=31, s_spread=True)
@@ -356,7 +357,7 @@ def _decode_case(B=3, Hq=4, Hkv=2, Lmax=64, d=8, seed=0):
     return q, kc, vc, g
 
 
-@pytest.mark.parametrize("gate_mode", [O.GATE_NONE, O.GATE_LOG_SOFTMAX])
+@pytest.mark.parametrize("gate_mode", [O.GATE_NONE, O.GATE_LOG_SOFTMAX, O.GATE_SOFTMAX_OUTSIDE])
 def test_decode_equals_last_prefill_row(gate_mode):
     """With L a multiple of the block, the decode query at position L−1 is the
     last row of the prefill forward with the same scores for its block."""
@@ -388,7 +389,7 @@ def test_decode_dense_ungated_ragged():
             assert np.abs(dec["o"][b, hq] - ref).max() < 1e-12
 
 
-@pytest.mark.parametrize("gate_mode", [O.GATE_NONE, O.GATE_LOG_SOFTMAX])
+@pytest.mark.parametrize("gate_mode", [O.GATE_NONE, O.GATE_LOG_SOFTMAX, O.GATE_SOFTMAX_OUTSIDE])
 def test_decode_split_invariance(gate_mode):
     """Merging split partials by their LSE gives the unsplit answer for any split count."""
     blk, Lmax, d = 8, 80, 8
@@ -459,7 +460,7 @@ def test_paged_decode_is_attention_over_the_gathered_pages():
             assert np.abs(dec["o"][b, hq] - ref).max() < 1e-12
 
 
-@pytest.mark.parametrize("gate_mode", [O.GATE_NONE, O.GATE_LOG_SOFTMAX])
+@pytest.mark.parametrize("gate_mode", [O.GATE_NONE, O.GATE_LOG_SOFTMAX, O.GATE_SOFTMAX_OUTSIDE])
 def test_paged_decode_equals_dense_decode(gate_mode):
     """Selection and gates too: the paged step gives the dense step's answer."""
     blk, Lmax, d = 8, 96, 8
@@ -554,3 +555,77 @@ def test_scored_selection_without_history():
     k = np.ones((2, 2, 128, 8))
     s, idx, lse = O.decode_select_scored(q, O.block_mean_keys(k), np.array([1, 64]), K=3)
     assert (idx == -1).all() and np.isneginf(lse).all() and np.isnan(s).all()
+
+
+# ---------------------------------------------------------------------------
+# The gate outside the softmax
+# ---------------------------------------------------------------------------
+def test_outside_gate_is_reweighted_dense_attention():
+    """Constant s and K covering the history give g_m = 1/t on every history block.
+    The output is then the current block's share of dense attention plus 1/t times
+    the history's share. The shares come from torch SDPA over each part and the
+    log-sum-exp of each part's logits."""
+    blk, N, d = 4, 32, 8
+    g = np.random.default_rng(77)
+    q = g.standard_normal((1, 2, N, d))
+    k = g.standard_normal((1, 1, N, d))
+    v = g.standard_normal((1, 1, N, d))
+    nb = N // blk
+    s = np.zeros((1, 1, nb, nb))
+    idx, _ = O.prefill_select(s, nb)
+    o, _ = O.forward(q, k, v, s, idx, block=blk, gate_mode=O.GATE_SOFTMAX_OUTSIDE)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    scale = 1 / math.sqrt(d)
+    for t in range(1, nb):
+        cur = slice(blk * t, blk * t + blk)
+        qb = tq[0, :, cur]  # [2, blk, d]
+        kc_, vc_ = tk[0, 0, cur], tv[0, 0, cur]
+        kh, vh = tk[0, 0, :blk * t], tv[0, 0, :blk * t]
+        causal = torch.ones(blk, blk, dtype=torch.bool).tril()
+        o_cur = torch.nn.functional.scaled_dot_product_attention(qb, kc_[None], vc_[None], attn_mask=causal)
+        o_hist = torch.nn.functional.scaled_dot_product_attention(qb, kh[None], vh[None])
+        z_cur = (qb @ kc_.T * scale).masked_fill(~causal, -math.inf)
+        z_hist = qb @ kh.T * scale
+        lse_cur = torch.logsumexp(z_cur, -1, keepdim=True)
+        lse_all = torch.logsumexp(torch.cat([z_cur, z_hist], -1), -1, keepdim=True)
+        w_cur = torch.exp(lse_cur - lse_all)
+        ref = w_cur * o_cur + (1 - w_cur) * o_hist / t
+        assert np.abs(o[0, :, cur] - ref.numpy()).max() < 1e-12, t
+
+
+def test_outside_gate_with_one_history_block_is_plain_attention():
+    """With one history block, g = softmax of one score = 1, inside or outside."""
+    q, k, v, do, s = _rand_case(B=1, Hq=2, Hkv=1, N=16, d=4, block=4, seed=78)
+    idx, _ = O.prefill_select(s, 2)
+    o4, L4 = O.forward(q, k, v, s, idx, block=4, gate_mode=O.GATE_SOFTMAX_OUTSIDE)
+    o1, L1 = O.forward(q, k, v, s, idx, block=4, gate_mode=O.GATE_NONE)
+    assert np.abs(o4[:, :, :8] - o1[:, :, :8]).max() < 1e-14
+    assert np.abs(L4 - L1).max() < 1e-12  # L is over the plain logits for every query block
+    assert np.abs(o4[:, :, 8:] - o1[:, :, 8:]).max() > 1e-3  # two history blocks: g < 1 matters
+
+
+def test_outside_gate_dl_matches_pages_formula():
+    """dl = g·dg, with the page's outside-gate gradient dg_m = Σ p_i dOᵀ v_i over the
+    tokens i of block m, summed over the block's rows and the group's heads. p is the
+    softmax over the plain logits, from torch."""
+    blk, N, d, K = 4, 24, 4, 3
+    q, k, v, do, s = _rand_case(B=1, Hq=2, Hkv=1, N=N, d=d, block=blk, seed=79)
+    idx, _ = O.prefill_select(s, K)
+    _, _, _, _, dl = O.backward(q, k, v, s, idx, do, block=blk, gate_mode=O.GATE_SOFTMAX_OUTSIDE)
+    scale = 1 / math.sqrt(d)
+    for t in range(1, N // blk):
+        sel = [int(m) for m in idx[0, 0, t] if m >= 0]
+        tok = np.concatenate([np.arange(blk * t, blk * t + blk)] + [np.arange(blk * m, blk * m + blk) for m in sel])
+        hist = s[0, 0, t, :t]
+        gate = np.exp(hist - np.log(np.exp(hist).sum()))
+        for slot, m in enumerate(sel):
+            dg = 0.0
+            for hq in range(2):
+                for i in range(blk * t, blk * t + blk):
+                    z = torch.from_numpy(scale * (k[0, 0, tok] @ q[0, hq, i]))
+                    z[:blk][np.arange(blk) > i - blk * t] = -math.inf  # causal inside the current block
+                    p = torch.softmax(z, 0).numpy()
+                    for jj, j in enumerate(tok):
+                        if blk * m <= j < blk * m + blk:
+                            dg += p[jj] * float(do[0, hq, i] @ v[0, 0, j])
+            assert abs(dl[0, 0, t, slot] - gate[m] * dg) < 1e-12, (t, slot)
