@@ -326,6 +326,56 @@ SAS_API sas_status sas_decode_noalloc(const sas_params* p, const sas_bf16* q, co
                                       void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Training steps end to end from host memory. The pages have no counterpart:
+ * this is the library's I/O path for callers whose batches live on the host.
+ * ------------------------------------------------------------------------- */
+
+/* One step's host buffers (pinned memory, for the copies to overlap; pageable
+ * memory works but serialises them). Inputs as in sas_fwd / sas_bwd; outputs
+ * as those calls write them. lse_o may be NULL (not copied back). ds must be
+ * NULL under SAS_GATE_NONE and may be NULL otherwise (not copied back). */
+typedef struct {
+  const sas_bf16* q;   /* [B, Hq, N, d] */
+  const sas_bf16* k;   /* [B, Hkv, N, d] */
+  const sas_bf16* v;   /* [B, Hkv, N, d] */
+  const float* s;      /* [B, Hkv, NQB, NKB] */
+  const sas_bf16* dO;  /* [B, Hq, N, d] */
+  sas_bf16* o;         /* [B, Hq, N, d] */
+  float* lse_o;        /* [B, Hq, N] or NULL */
+  sas_bf16* dq;        /* [B, Hq, N, d] */
+  sas_bf16* dk;        /* [B, Hkv, N, d] */
+  sas_bf16* dv;        /* [B, Hkv, N, d] */
+  float* ds;           /* [B, Hkv, NQB, NKB] or NULL */
+} sas_host_step;
+
+/* One set of caller-owned device buffers for a step, with the layouts of the
+ * host buffers, plus idx int32 [B, Hkv, NQB, K], lse_s fp32 [B, Hkv, NQB], and
+ * the backward workspace (sas_bwd_workspace_size bytes, 256-byte aligned). ds
+ * is required under every gate mode but SAS_GATE_NONE. */
+typedef struct {
+  sas_bf16 *q, *k, *v, *dO, *o, *dq, *dk, *dv;
+  float *s, *lse_s, *lse_o, *ds;
+  int32_t* idx;
+  void* ws;
+  size_t ws_bytes;
+} sas_device_slot;
+
+/* Runs n_steps training steps (select + LSE, forward, backward with ds), step
+ * i on device slot i % 2 (slots[0..1]; one slot is enough when n_steps = 1).
+ * Step i's inputs are copied from steps[i] to the slot, its kernels run on
+ * `stream`, and its outputs are copied back to steps[i]. The upload of step
+ * i + 1 and the download of step i − 1 run on two internal copy streams while
+ * step i's kernels run. The call is asynchronous: when `stream` has completed,
+ * every step's outputs are in host memory. Host buffers may be shared between
+ * steps (the copies of one direction run in step order), but a step's host
+ * outputs must not be read before `stream` completes.
+ * Errors: the argument checks of sas_fwd and sas_bwd for every slot and step,
+ * before anything is enqueued (SAS_ERR_INVALID_ARG, SAS_ERR_WORKSPACE);
+ * SAS_ERR_CUDA if a copy or launch cannot be enqueued. */
+SAS_API sas_status sas_train_steps_host(const sas_params* p, int n_steps, const sas_host_step* steps,
+                                        const sas_device_slot* slots, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Diagnostics
  * ------------------------------------------------------------------------- */
 

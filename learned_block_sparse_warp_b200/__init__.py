@@ -26,7 +26,7 @@ __all__ = [
     "sas_decode_combine", "sas_decode_paged", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string",
     "sas_version",
     "DecodeGraph", "sas_selftest_wait_timeout", "sas_block_mean_keys", "sas_decode_select_scored",
-    "decode_step_scored",
+    "decode_step_scored", "sas_train_steps_host", "empty_device_slot",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
@@ -44,6 +44,17 @@ class SasError(RuntimeError):
     def __init__(self, fn: str, code: int):
         self.code = code
         super().__init__(f"{fn} failed: {sas_status_string(code)}")
+
+
+class sas_host_step(ctypes.Structure):
+    """Mirror of ``sas_host_step``: one training step's host buffers."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("q", "k", "v", "s", "dO", "o", "lse_o", "dq", "dk", "dv", "ds")]
+
+
+class sas_device_slot(ctypes.Structure):
+    """Mirror of ``sas_device_slot``: one set of device buffers for a step."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("q", "k", "v", "dO", "o", "dq", "dk", "dv", "s", "lse_s", "lse_o",
+                                                "ds", "idx", "ws")] + [("ws_bytes", ctypes.c_size_t)]
 
 
 class sas_params(ctypes.Structure):
@@ -74,6 +85,7 @@ def _load() -> ctypes.CDLL:
         "sas_selftest_wait_timeout": [vp],
         "sas_block_mean_keys": [P, vp, vp, vp, vp],
         "sas_decode_select_scored": [P, vp, vp, vp, vp, vp, vp, vp],
+        "sas_train_steps_host": [P, ctypes.c_int, ctypes.POINTER(sas_host_step), ctypes.POINTER(sas_device_slot), vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -264,6 +276,44 @@ def sas_decode_select_scored(p: Params, q, kmean, cache_len, s, idx, lse_s=None,
         _ptr(lse_s, f32, sh["lse_s"], "lse_s"), _stream(stream)))
 
 
+def _host_ptr(t: Optional[torch.Tensor], dtype, shape, name: str):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError(f"{name}: expected a host tensor (pinned memory lets the copies overlap)")
+    if not t.is_contiguous() or t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected a contiguous {dtype} tensor of shape {tuple(shape)}")
+    return t.data_ptr()
+
+
+def sas_train_steps_host(p: Params, steps, slots, stream=None) -> None:
+    """Training steps end to end from host memory (see include/sas.h): step i runs on slots[i % 2],
+    with the upload of step i + 1 and the download of step i - 1 overlapping step i's kernels.
+
+    steps: list of dicts of host tensors with keys q, k, v, s, do (inputs) and o, lse_o, dq, dk, dv,
+    ds (outputs; lse_o and ds may be missing). slots: one or two dicts from ``empty_device_slot``.
+    Asynchronous on ``stream``."""
+    B, Hq, Hkv, N, d, NB = p.batch, p.n_q_heads, p.n_kv_heads, p.seq_len, p.head_dim, p.n_blocks
+    qs, kvs, ss, ls = (B, Hq, N, d), (B, Hkv, N, d), (B, Hkv, NB, NB), (B, Hq, N)
+    hs = (sas_host_step * len(steps))()
+    for i, st in enumerate(steps):
+        hs[i] = sas_host_step(
+            _host_ptr(st["q"], bf16, qs, "q"), _host_ptr(st["k"], bf16, kvs, "k"), _host_ptr(st["v"], bf16, kvs, "v"),
+            _host_ptr(st["s"], f32, ss, "s"), _host_ptr(st["do"], bf16, qs, "do"), _host_ptr(st["o"], bf16, qs, "o"),
+            _host_ptr(st.get("lse_o"), f32, ls, "lse_o"), _host_ptr(st["dq"], bf16, qs, "dq"),
+            _host_ptr(st["dk"], bf16, kvs, "dk"), _host_ptr(st["dv"], bf16, kvs, "dv"),
+            _host_ptr(st.get("ds"), f32, ss, "ds"))
+    ds_ = (sas_device_slot * 2)()
+    for k, sl in enumerate(slots[:2]):
+        ptr = {n: (_ptr(sl[n]).value if sl.get(n) is not None else None) for n in
+               ("q", "k", "v", "do", "o", "dq", "dk", "dv", "s", "lse_s", "lse_o", "ds", "idx", "ws")}
+        ds_[k] = sas_device_slot(ptr["q"], ptr["k"], ptr["v"], ptr["do"], ptr["o"], ptr["dq"], ptr["dk"], ptr["dv"],
+                                 ptr["s"], ptr["lse_s"], ptr["lse_o"], ptr["ds"], ptr["idx"], ptr["ws"],
+                                 sl["ws"].numel() if sl.get("ws") is not None else 0)
+    _check("sas_train_steps_host", lib.sas_train_steps_host(ctypes.byref(p.c()), len(steps), hs, ds_,
+                                                            _stream(stream)))
+
+
 def sas_selftest_wait_timeout(stream=None) -> None:
     """One bounded wait that runs out (about a second); sas_get_device_error then reads SAS_ERR_TIMEOUT."""
     _check("sas_selftest_wait_timeout", lib.sas_selftest_wait_timeout(_stream(stream)))
@@ -295,6 +345,18 @@ def empty_prefill_outputs(p: Params, device="cuda", backward: bool = True) -> di
             ws=torch.empty((sas_bwd_workspace_size(p),), dtype=torch.uint8, device=device),
         )
     return out
+
+
+def empty_device_slot(p: Params, device="cuda") -> dict:
+    """Device buffers of one training step for ``sas_train_steps_host``: inputs, outputs, idx, lse_s, workspace."""
+    B, Hq, Hkv, N, d, NB = p.batch, p.n_q_heads, p.n_kv_heads, p.seq_len, p.head_dim, p.n_blocks
+    slot = dict(q=torch.empty((B, Hq, N, d), dtype=bf16, device=device),
+                k=torch.empty((B, Hkv, N, d), dtype=bf16, device=device),
+                v=torch.empty((B, Hkv, N, d), dtype=bf16, device=device),
+                s=torch.empty((B, Hkv, NB, NB), dtype=f32, device=device),
+                do=torch.empty((B, Hq, N, d), dtype=bf16, device=device))
+    slot.update(empty_prefill_outputs(p, device=device, backward=True))
+    return slot
 
 
 def empty_decode_outputs(p: Params, n_split: int, device="cuda") -> dict:

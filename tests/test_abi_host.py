@@ -202,3 +202,68 @@ def test_decode_select_scored_checked():
     # a row of more than 8 x 53,248 history blocks does not fit a cluster's shared memory
     big = _p(n_q_heads=1, n_kv_heads=1, seq_len=64 * (8 * 53248 + 2)).c()
     assert call(params=big) == UNSUPPORTED
+
+
+def test_host_step_structs_match_the_header():
+    """Field order and size of sas_host_step / sas_device_slot, compiled from the header by gcc."""
+    import subprocess
+    import tempfile
+    src = r'''
+#include <stddef.h>
+#include <stdio.h>
+#include "sas.h"
+#define F(T, m) printf("%s %zu\n", #m, offsetof(T, m));
+int main(void) {
+  printf("host %zu\n", sizeof(sas_host_step));
+  F(sas_host_step, q) F(sas_host_step, k) F(sas_host_step, v) F(sas_host_step, s) F(sas_host_step, dO)
+  F(sas_host_step, o) F(sas_host_step, lse_o) F(sas_host_step, dq) F(sas_host_step, dk) F(sas_host_step, dv)
+  F(sas_host_step, ds)
+  printf("slot %zu\n", sizeof(sas_device_slot));
+  F(sas_device_slot, q) F(sas_device_slot, k) F(sas_device_slot, v) F(sas_device_slot, dO) F(sas_device_slot, o)
+  F(sas_device_slot, dq) F(sas_device_slot, dk) F(sas_device_slot, dv) F(sas_device_slot, s)
+  F(sas_device_slot, lse_s) F(sas_device_slot, lse_o) F(sas_device_slot, ds) F(sas_device_slot, idx)
+  F(sas_device_slot, ws) F(sas_device_slot, ws_bytes)
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as tmp:
+        c = os.path.join(tmp, "layout.c")
+        exe = os.path.join(tmp, "layout")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-std=c11", f"-I{os.path.join(ROOT, 'include')}", c, "-o", exe], check=True)
+        lines = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = dict(ln.split() for ln in lines if ln)
+    assert int(got["host"]) == ctypes.sizeof(sas.sas_host_step)
+    assert int(got["slot"]) == ctypes.sizeof(sas.sas_device_slot)
+    host_off = [getattr(sas.sas_host_step, n).offset for n, _ in sas.sas_host_step._fields_]
+    slot_off = [getattr(sas.sas_device_slot, n).offset for n, _ in sas.sas_device_slot._fields_]
+    vals = [int(v) for k, v in (ln.split() for ln in lines if ln) if k not in ("host", "slot")]
+    assert vals == host_off + slot_off
+
+
+def test_train_steps_host_checked():
+    p = _p()
+    c = p.c()
+    n = sas.sas_bwd_workspace_size(p)
+    slot = sas.sas_device_slot(*([A] * 14), n)
+    step = sas.sas_host_step(*([A] * 11))
+    slots = (sas.sas_device_slot * 2)(slot, slot)
+    steps = (sas.sas_host_step * 3)(step, step, step)
+    f = lib.sas_train_steps_host
+    assert f(None, 3, steps, slots, None) == INVALID
+    assert f(ctypes.byref(c), 0, steps, slots, None) == INVALID
+    assert f(ctypes.byref(c), 3, None, slots, None) == INVALID
+    assert f(ctypes.byref(c), 3, steps, None, None) == INVALID
+    small = (sas.sas_device_slot * 2)(slot, sas.sas_device_slot(*([A] * 14), n - 1))
+    assert f(ctypes.byref(c), 3, steps, small, None) == WORKSPACE
+    bad_slot = (sas.sas_device_slot * 2)(slot, sas.sas_device_slot(*([A] * 13), None, n))
+    assert f(ctypes.byref(c), 3, steps, bad_slot, None) == WORKSPACE
+    no_dq = sas.sas_device_slot(*([A] * 14), n)
+    no_dq.dq = None
+    assert f(ctypes.byref(c), 3, steps, (sas.sas_device_slot * 2)(slot, no_dq), None) == INVALID
+    bad_step = sas.sas_host_step(*([A] * 11))
+    bad_step.dO = None
+    assert f(ctypes.byref(c), 3, (sas.sas_host_step * 3)(step, step, bad_step), slots, None) == INVALID
+    # no ds without a gate
+    c_none = _p(gate_mode=1).c()
+    assert f(ctypes.byref(c_none), 3, steps, slots, None) == INVALID
