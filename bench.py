@@ -444,6 +444,15 @@ def run_gpu(args, rank, world, local_rank):
         if sas.sas_get_device_error(stream) != 0:
             raise RuntimeError("device error during decode")
 
+    # ---------------- the 128K forward and the budget x length sweep ----------------
+    if args.only in ("all", "sweep"):
+        try:
+            line["sweep"] = sweep_section(args, sas, stream, dev, pk, dist, world)
+        except Exception as e:  # a supplementary section: its failure is reported, not the whole line lost
+            if args.only == "sweep":
+                raise
+            line["sweep"] = {"error": f"{type(e).__name__}: {e}"[:400]}
+
     # ---------------- long-context decode that scores its own history ----------------
     if args.only in ("all", "long_decode") and not args.no_decode:
         try:
@@ -458,6 +467,94 @@ def run_gpu(args, rank, world, local_rank):
     if dist is not None:
         dist.destroy_process_group()
     return line
+
+
+# ---------------------------------------------------------------------------
+# the Llama-3.1-8B 128K forward and the Qwen3-14B budget x length sweep
+# ---------------------------------------------------------------------------
+SWEEP = ["llama31_8b_fwd_128k"] + [f"qwen3_14b_k{k}_n{n}" for k in (16, 32, 64) for n in (8192, 32768, 65536)]
+
+
+def sweep_inputs(w, dev, torch):
+    """Seeded device-side inputs with the workload's recipe: q, k, v, dO ~ N(0, 1) bf16, and s ~ N(0, 2),
+    or, with heavy hitters, s = block-mean(k) . block-and-group-mean(q) / sqrt(d) + N(0, 0.5) after
+    1% of the keys and every query of the group get 4 u_h."""
+    B, Hq, Hkv, N, d, NB, G = w.batch, w.n_q_heads, w.n_kv_heads, w.seq_len, w.head_dim, w.n_blocks, w.group
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    bf = torch.bfloat16
+    q = torch.randn((B, Hq, N, d), generator=gen, device=dev, dtype=torch.float32)
+    k = torch.randn((B, Hkv, N, d), generator=gen, device=dev, dtype=torch.float32)
+    if w.heavy_hitters:
+        u = torch.randn((B, Hkv, d), generator=gen, device=dev)
+        u = u / u.norm(dim=-1, keepdim=True)
+        n_hh = max(1, round(0.01 * N))
+        for b in range(B):
+            for h in range(Hkv):
+                pos = torch.randperm(N, generator=gen, device=dev)[:n_hh]
+                k[b, h, pos] += 4 * u[b, h]
+        q += 4 * u.repeat_interleave(G, dim=1)[:, :, None, :]
+    q, k = q.to(bf), k.to(bf)
+    v = torch.randn((B, Hkv, N, d), generator=gen, device=dev, dtype=torch.float32).to(bf)
+    if w.heavy_hitters:
+        kbar = k.float().view(B, Hkv, NB, 64, d).mean(3)
+        qbar = q.float().view(B, Hkv, G, NB, 64, d).mean((2, 4))
+        s = qbar @ kbar.transpose(-1, -2) / math.sqrt(d)
+        s += math.sqrt(0.5) * torch.randn(s.shape, generator=gen, device=dev)
+    else:
+        s = math.sqrt(w.s_var) * torch.randn((B, Hkv, NB, NB), generator=gen, device=dev)
+    x = dict(q=q, k=k, v=v, s=s.contiguous())
+    if w.backward:
+        x["do"] = torch.randn((B, Hq, N, d), generator=gen, device=dev, dtype=torch.float32).to(bf)
+    return x
+
+
+def sweep_section(args, sas, stream, dev, pk, dist, world):
+    import torch
+    from synth import workloads as W
+    points = []
+    for name in SWEEP:
+        w = W.WORKLOADS[name]
+        p = sas.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
+                       seq_len=w.seq_len, top_k=w.top_k, gate_mode=sas.SAS_GATE_LOG_SOFTMAX)
+        with torch.cuda.stream(stream):
+            x = sweep_inputs(w, dev, torch)
+        torch.cuda.synchronize()
+        out = sas.empty_prefill_outputs(p, device=dev, backward=w.backward)
+
+        def run():
+            sas.prefill_step(p, x["q"], x["k"], x["v"], x["s"], x.get("do"), out, backward=w.backward,
+                             stream=stream)
+
+        n = max(5, min(args.steps, 10))
+        with torch.cuda.stream(stream):
+            for _ in range(max(3, args.warmup)):
+                run()
+        torch.cuda.synchronize()
+        barrier(dist)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(n):
+                run()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if sas.sas_get_device_error(stream) != 0:
+            raise RuntimeError(f"device error in {name}")
+        ms = max_over_ranks(dist, a.elapsed_time(b), dev) / n
+        F = fwd_flops(w.n_q_heads, w.head_dim, w.n_blocks, w.top_k, batch=w.batch)
+        flops = (3.5 if w.backward else 1.0) * F
+        tf = job_rate(flops, world, ms * 1e-3) / 1e12
+        points.append({"workload": name, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "seq_len": w.seq_len,
+                       "top_k": w.top_k, "pass": "fwd+bwd" if w.backward else "fwd", "tflop_per_step": flops / 1e12,
+                       "ms_per_step": ms, "tflops": tf, "frac": tf / (pk["bf16_sustained"] * world)})
+        del x, out
+        torch.cuda.empty_cache()
+    return {"points": points, "peak": pk["bf16_sustained"], "peak_source": pk["source"] + " sustained bf16",
+            "gate": "log_softmax (training form)",
+            "data": "synthetic, from a seeded device generator with each workload's recipe",
+            "l2": "inputs larger than L2 at every point (no flush)"}
 
 
 # ---------------------------------------------------------------------------
@@ -594,7 +691,7 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sas", "reference"], default="sas")
-    ap.add_argument("--only", choices=["all", "train", "decode", "long_decode"], default="all",
+    ap.add_argument("--only", choices=["all", "train", "decode", "long_decode", "sweep"], default="all",
                     help="run only one workload (for profiling); the JSON line needs 'all'")
     ap.add_argument("--n-split", type=int, default=0, help="decode splits (0: K + 1)")
     ap.add_argument("--no-e2e", action="store_true")
