@@ -61,3 +61,28 @@ def test_decode_gathered_bytes():
         c = (int(L) - 1) // 64
         want += 8 * (min(16, c) * 64 + (int(L) - 64 * c)) * 128 * 2 * 2
     assert bench.decode_kv_bytes(w, lens) == want
+
+
+def test_bench_sections_name_real_workloads():
+    """The sweep and long-context sections look their workloads up by name and shape."""
+    for name in bench.SWEEP:
+        w = W.WORKLOADS[name]
+        assert w.kind == "prefill" and w.seq_len % 64 == 0
+    assert W.WORKLOADS["llama31_8b_fwd_128k"].backward is False and W.WORKLOADS["llama31_8b_fwd_128k"].heavy_hitters
+    assert all(W.WORKLOADS[n].backward for n in bench.SWEEP[1:])
+    for B, L in bench.LONG_DECODE:
+        assert B >= 1 and L % 64 == 0 and (L // 64 - 1 + 7) // 8 <= 53248  # fits the scored select's clusters
+    assert bench.TRAIN in W.WORKLOADS and bench.DECODE in W.WORKLOADS
+
+
+def test_sweep_inputs_follow_the_workload_recipe():
+    import torch
+    w = W.custom("hh", batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, seq_len=4096, top_k=8, seed=3,
+                 backward=False, heavy_hitters=True)
+    x = bench.sweep_inputs(w, torch.device("cpu"), torch)
+    assert set(x) == {"q", "k", "v", "s"} and x["s"].shape == (1, 2, 64, 64)
+    assert x["q"].dtype == torch.bfloat16 and x["s"].dtype == torch.float32
+    w2 = W.custom("plain", batch=1, n_q_heads=10, n_kv_heads=2, head_dim=128, seq_len=2048, top_k=8, seed=4)
+    x2 = bench.sweep_inputs(w2, torch.device("cpu"), torch)
+    assert set(x2) == {"q", "k", "v", "s", "do"}
+    assert abs(float(x2["s"].std()) - 2 ** 0.5) < 0.1  # s ~ N(0, 2)
