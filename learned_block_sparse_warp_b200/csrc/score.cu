@@ -28,6 +28,10 @@
 // lower-ranked CTA's slice first, and the chosen blocks are written in
 // ascending order. The selected set is exact: it is the one a full sort of the
 // kernel's scores picks.
+//
+// The same kernel with D = 0 reads the scores from s instead of computing
+// them. The decode form of sas_topk_select uses it for rows past 2048 blocks,
+// where one CTA or warp per row would walk the row 32 times.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -51,8 +55,8 @@ struct ScoredSelectArgs {
   const uint16_t* q;      // [B, Hq, d] bf16
   const uint16_t* kmean;  // [B, Hkv, NB, d] bf16
   const int32_t* cache_len;
-  float* s;               // [B, Hkv, NB]: entries m < c written
-  int32_t* idx;           // [B, Hkv, K]
+  float* s;               // [B, Hkv, NB]: entries m < c written (D > 0) or read (D = 0)
+  int32_t* idx;           // [B, Hkv, K], or null for LSE(s) alone
   float* lse;             // [B, Hkv] or null
   int* err;
   int Hq, Hkv, G, NB, K;
@@ -149,10 +153,11 @@ __device__ __forceinline__ uint32_t bins_incl_scan(uint32_t v, uint32_t* wsum) {
   return threadIdx.x < ssc::kBins ? v + before : 0u;
 }
 
+// D = 64 or 128: scores from q and k̄; D = 0: scores read from s.
 template <int D>
 __global__ void __launch_bounds__(ssc::kThreads) select_scored_kernel(ScoredSelectArgs a) {
   extern __shared__ float sc[];  // this CTA's slice of the row's scores
-  __shared__ float qbar[D];
+  __shared__ float qbar[D > 0 ? D : 1];
   __shared__ uint32_t hist[2][ssc::kBins];
   __shared__ float red[ssc::kWarps];
   __shared__ int wtot[ssc::kWarps];
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(ssc::kThreads) select_scored_kernel(ScoredSele
   const int b = row / a.Hkv, h = row - b * a.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  griddep_wait();  // q, k̄ and cache_len may come from the work just before this launch
+  griddep_wait();  // q, k̄ (or s) and cache_len may come from the work just before this launch
   griddep_launch_dependents();
   const int L = a.cache_len[b];
   int c = (L - 1) / kBlock;
@@ -178,6 +183,10 @@ __global__ void __launch_bounds__(ssc::kThreads) select_scored_kernel(ScoredSele
   const int per = (c + C - 1) / C;
   const int m0 = min(c, rank * per), m1 = min(c, m0 + per), n_loc = m1 - m0;
 
+  if constexpr (D == 0) {  // the given scores of blocks m0..m1-1
+    const float* srow = a.s + size_t(row) * a.NB + m0;
+    for (int i = tid; i < n_loc; i += ssc::kThreads) sc[i] = __ldg(srow + i);
+  } else {
   for (int i = tid; i < D; i += ssc::kThreads) {
     const uint16_t* qp = a.q + (size_t(b) * a.Hq + size_t(h) * a.G) * D + i;
     float acc = 0.f;
@@ -215,6 +224,7 @@ __global__ void __launch_bounds__(ssc::kThreads) select_scored_kernel(ScoredSele
       }
     }
   }
+  }  // scores computed
   __syncthreads();
 
   // ---- LSE(s) over the whole row ----
@@ -242,7 +252,9 @@ __global__ void __launch_bounds__(ssc::kThreads) select_scored_kernel(ScoredSele
   // ---- Top-K: n = min(K, c) blocks, ascending ----
   const int n = min(a.K, c);
   int32_t* irow = a.idx + size_t(row) * a.K;
-  if (n == c) {
+  if (a.idx == nullptr) {
+    // LSE(s) alone
+  } else if (n == c) {
     for (int m = m0 + tid; m < m1; m += ssc::kThreads) irow[m] = m;
   } else {
     // Radix select of the n-th largest key, 8 bits a pass from the top. After
@@ -323,7 +335,7 @@ __global__ void __launch_bounds__(ssc::kThreads) select_scored_kernel(ScoredSele
       eq_seen += e_tot;
     }
   }
-  if (rank == 0)
+  if (rank == 0 && a.idx != nullptr)
     for (int k = n + tid; k < a.K; k += ssc::kThreads) irow[k] = -1;
   cluster.sync();  // no CTA leaves while another may still read its shared memory
 }
@@ -417,6 +429,23 @@ int scored_cluster_size(int rows, int NB, int sms) {
   return (hist + C - 1) / C > ssc::kMaxSlice ? 0 : C;
 }
 
+// SM count of the current device, fetched once per device (a benign race:
+// every writer stores the same value).
+static cudaError_t device_sm_count(int* out) {
+  static int sm_count[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (sm_count[dev] == 0) {
+    int n = 0;
+    if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    sm_count[dev] = n;
+  }
+  *out = sm_count[dev];
+  return cudaSuccess;
+}
+
 template <int D>
 static cudaError_t launch_scored_d(const ScoredSelectArgs& a, int rows, int C, cudaStream_t st) {
   const int slice = (a.NB - 1 + C - 1) / C;
@@ -444,17 +473,9 @@ static cudaError_t launch_scored_d(const ScoredSelectArgs& a, int rows, int C, c
 cudaError_t launch_select_scored(const Shape& sh, const uint16_t* q, const uint16_t* kmean,
                                  const int32_t* cache_len, float* s, int32_t* idx, float* lse, int* err,
                                  cudaStream_t st) {
-  static int sm_count[64];  // per device, fetched once (a benign race: every writer stores the same value)
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  int sms = 0;
+  cudaError_t e = device_sm_count(&sms);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (sm_count[dev] == 0) {
-    int n = 0;
-    if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    sm_count[dev] = n;
-  }
-  const int sms = sm_count[dev];
   const int rows = sh.B * sh.Hkv;
   const int C = scored_cluster_size(rows, sh.NB, sms);
   if (C == 0) return cudaErrorInvalidValue;  // the host entry rules this out first
@@ -462,6 +483,20 @@ cudaError_t launch_select_scored(const Shape& sh, const uint16_t* q, const uint1
                      sh.scale / float(sh.G)};
   if (sh.d == 128) return launch_scored_d<128>(a, rows, C, st);
   return launch_scored_d<64>(a, rows, C, st);
+}
+
+// The decode form of sas_topk_select on given scores, one cluster per row.
+cudaError_t launch_select_cluster(const Shape& sh, const float* s, const int32_t* cache_len, int32_t* idx,
+                                  float* lse, int* err, cudaStream_t st) {
+  int sms = 0;
+  cudaError_t e = device_sm_count(&sms);
+  if (e != cudaSuccess) return e;
+  const int rows = sh.B * sh.Hkv;
+  const int C = scored_cluster_size(rows, sh.NB, sms);
+  if (C == 0) return cudaErrorInvalidValue;
+  ScoredSelectArgs a{nullptr, nullptr, cache_len, const_cast<float*>(s), idx, lse, err, sh.Hq, sh.Hkv, sh.G,
+                     sh.NB, sh.K, 0.f};
+  return launch_scored_d<0>(a, rows, C, st);
 }
 
 }  // namespace sas

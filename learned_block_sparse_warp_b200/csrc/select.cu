@@ -11,6 +11,8 @@
 // at the threshold from the lowest block index, then writes the chosen blocks
 // in ascending order with ballots. The row stays in L1 across the passes.
 // Every selected set is exact, so the result matches a full sort bit for bit.
+// Decode rows of up to 2048 blocks take one CTA each; longer decode rows go to
+// the cluster radix select of score.cu.
 #include "common.cuh"
 
 namespace sas {
@@ -326,8 +328,15 @@ static void launch_select_r(const Shape& sh, const float* s, const int32_t* cach
   }
 }
 
+bool scored_rows_fit(int NB);
+cudaError_t launch_select_cluster(const Shape& sh, const float* s, const int32_t* cache_len, int32_t* idx,
+                                  float* lse, int* err, cudaStream_t st);
+
 cudaError_t launch_select(const Shape& sh, const float* s, const int32_t* cache_len, int32_t* idx, float* lse,
                           int* err, cudaStream_t st) {
+  // decode rows past 2048 blocks: a radix select over a cluster of CTAs per row
+  if (cache_len != nullptr && sh.NB > kRowThreads * kRowSlots && scored_rows_fit(sh.NB))
+    return launch_select_cluster(sh, s, cache_len, idx, lse, err, st);
   // rows hold at most NB - 1 history scores
   if (sh.NB <= 4 * 32) launch_select_r<4>(sh, s, cache_len, idx, lse, err, st);
   else if (sh.NB <= 16 * 32) launch_select_r<16>(sh, s, cache_len, idx, lse, err, st);
