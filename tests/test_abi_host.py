@@ -267,3 +267,36 @@ def test_train_steps_host_checked():
     # no ds without a gate
     c_none = _p(gate_mode=1).c()
     assert f(ctypes.byref(c_none), 3, steps, slots, None) == INVALID
+
+
+def test_plain_c_program_links_the_library():
+    """The boundary is usable from C alone: compile against include/sas.h, link libsas_b200.so and
+    call the entry points that need no GPU (version, status strings, workspace size, argument checks)."""
+    import subprocess
+    import tempfile
+    src = r'''
+#include <stdio.h>
+#include "sas.h"
+int main(void) {
+  sas_params p = {1, 8, 2, 128, 1024, 64, 4, 0.0f, SAS_GATE_LOG_SOFTMAX};
+  size_t ws = 0;
+  if (sas_bwd_workspace_size(&p, &ws) != SAS_OK || ws == 0) return 1;
+  if (sas_fwd(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL) != SAS_ERR_INVALID_ARG) return 2;
+  p.head_dim = 96;
+  if (sas_bwd_workspace_size(&p, &ws) != SAS_ERR_UNSUPPORTED) return 3;
+  printf("%d %zu %s\n", sas_version(), ws, sas_status_string(SAS_ERR_TIMEOUT));
+  return 0;
+}
+'''
+    lib_dir = os.path.dirname(sas.LIB_PATH)
+    with tempfile.TemporaryDirectory() as tmp:
+        c = os.path.join(tmp, "use_sas.c")
+        exe = os.path.join(tmp, "use_sas")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-std=c11", f"-I{os.path.join(ROOT, 'include')}", c, f"-L{lib_dir}", "-l:libsas_b200.so",
+                        f"-Wl,-rpath,{lib_dir}", "-o", exe], check=True)
+        r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    ver, ws, msg = r.stdout.split(maxsplit=2)
+    assert int(ver) == sas.sas_version() and int(ws) == sas.sas_bwd_workspace_size(_p(n_q_heads=8, n_kv_heads=2))
+    assert msg.startswith("SAS_ERR_TIMEOUT")
