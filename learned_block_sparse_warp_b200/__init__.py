@@ -303,10 +303,14 @@ def sas_train_steps_host(p: Params, steps, slots, stream=None) -> None:
             _host_ptr(st.get("lse_o"), f32, ls, "lse_o"), _host_ptr(st["dq"], bf16, qs, "dq"),
             _host_ptr(st["dk"], bf16, kvs, "dk"), _host_ptr(st["dv"], bf16, kvs, "dv"),
             _host_ptr(st.get("ds"), f32, ss, "ds"))
+    K = p.top_k
+    slot_layout = dict(q=(bf16, qs), k=(bf16, kvs), v=(bf16, kvs), do=(bf16, qs), o=(bf16, qs), dq=(bf16, qs),
+                       dk=(bf16, kvs), dv=(bf16, kvs), s=(f32, ss), lse_s=(f32, (B, Hkv, NB)), lse_o=(f32, ls),
+                       ds=(f32, ss), idx=(i32, (B, Hkv, NB, K)), ws=(torch.uint8, None))
     ds_ = (sas_device_slot * 2)()
     for k, sl in enumerate(slots[:2]):
-        ptr = {n: (_ptr(sl[n]).value if sl.get(n) is not None else None) for n in
-               ("q", "k", "v", "do", "o", "dq", "dk", "dv", "s", "lse_s", "lse_o", "ds", "idx", "ws")}
+        ptr = {n: (_ptr(sl[n], dt, shp, f"slots[{k}].{n}").value if sl.get(n) is not None else None)
+               for n, (dt, shp) in slot_layout.items()}
         ds_[k] = sas_device_slot(ptr["q"], ptr["k"], ptr["v"], ptr["do"], ptr["o"], ptr["dq"], ptr["dk"], ptr["dv"],
                                  ptr["s"], ptr["lse_s"], ptr["lse_o"], ptr["ds"], ptr["idx"], ptr["ws"],
                                  sl["ws"].numel() if sl.get("ws") is not None else 0)
