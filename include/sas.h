@@ -371,7 +371,9 @@ typedef struct {
  * outputs must not be read before `stream` completes.
  * Errors: the argument checks of sas_fwd and sas_bwd for every slot and step,
  * before anything is enqueued (SAS_ERR_INVALID_ARG, SAS_ERR_WORKSPACE);
- * SAS_ERR_CUDA if a copy or launch cannot be enqueued. */
+ * SAS_ERR_CUDA if a copy or launch cannot be enqueued. After such an error
+ * the caller's stream still waits for every copy already enqueued, so buffers
+ * may be released once it completes. */
 SAS_API sas_status sas_train_steps_host(const sas_params* p, int n_steps, const sas_host_step* steps,
                                         const sas_device_slot* slots, void* stream);
 

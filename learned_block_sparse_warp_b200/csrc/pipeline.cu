@@ -80,29 +80,39 @@ extern "C" sas_status sas_train_steps_host(const sas_params* p, int n_steps, con
   if (e == cudaSuccess) e = cudaStreamWaitEvent(cr.down, cr.entry, 0);
   if (e != cudaSuccess) return SAS_ERR_CUDA;
   const cudaMemcpyKind H2D = cudaMemcpyHostToDevice, D2H = cudaMemcpyDeviceToHost;
+  // Every return after this point first makes the caller's stream wait for whatever the copy
+  // streams hold, so that no copy is still in flight once the caller's stream has completed.
+  auto leave = [&](sas_status status) {
+    cudaEvent_t j = nullptr;
+    bool joined = cudaEventCreateWithFlags(&j, cudaEventDisableTiming) == cudaSuccess;
+    for (cudaStream_t cp : {cr.up, cr.down})
+      joined = joined && cudaEventRecord(j, cp) == cudaSuccess && cudaStreamWaitEvent(cs, j, 0) == cudaSuccess;
+    if (j != nullptr) cudaEventDestroy(j);
+    return joined ? status : (status == SAS_OK ? SAS_ERR_CUDA : status);
+  };
 
   for (int i = 0; i < n_steps; ++i) {
     const int k = i & 1;
     const sas_device_slot& d = slots[k];
     const sas_host_step& h = steps[i];
     // inputs into slot k, once the kernels of step i − 2 have read them
-    if (i >= 2 && (e = cudaStreamWaitEvent(cr.up, cr.done[k], 0)) != cudaSuccess) return SAS_ERR_CUDA;
+    if (i >= 2 && (e = cudaStreamWaitEvent(cr.up, cr.done[k], 0)) != cudaSuccess) return leave(SAS_ERR_CUDA);
     if ((e = cudaMemcpyAsync(d.q, h.q, b_q, H2D, cr.up)) != cudaSuccess ||
         (e = cudaMemcpyAsync(d.k, h.k, b_kv, H2D, cr.up)) != cudaSuccess ||
         (e = cudaMemcpyAsync(d.v, h.v, b_kv, H2D, cr.up)) != cudaSuccess ||
         (e = cudaMemcpyAsync(d.s, h.s, b_s, H2D, cr.up)) != cudaSuccess ||
         (e = cudaMemcpyAsync(d.dO, h.dO, b_q, H2D, cr.up)) != cudaSuccess ||
         (e = cudaEventRecord(cr.in[k], cr.up)) != cudaSuccess)
-      return SAS_ERR_CUDA;
+      return leave(SAS_ERR_CUDA);
     // kernels, once the inputs have landed and the outputs of step i − 2 have left
-    if ((e = cudaStreamWaitEvent(cs, cr.in[k], 0)) != cudaSuccess) return SAS_ERR_CUDA;
-    if (i >= 2 && (e = cudaStreamWaitEvent(cs, cr.out[k], 0)) != cudaSuccess) return SAS_ERR_CUDA;
-    if ((r = sas_topk_select(p, d.s, nullptr, d.idx, d.lse_s, stream)) != SAS_OK) return r;
-    if ((r = sas_fwd(p, d.q, d.k, d.v, d.s, d.idx, d.lse_s, d.o, d.lse_o, stream)) != SAS_OK) return r;
+    if ((e = cudaStreamWaitEvent(cs, cr.in[k], 0)) != cudaSuccess) return leave(SAS_ERR_CUDA);
+    if (i >= 2 && (e = cudaStreamWaitEvent(cs, cr.out[k], 0)) != cudaSuccess) return leave(SAS_ERR_CUDA);
+    if ((r = sas_topk_select(p, d.s, nullptr, d.idx, d.lse_s, stream)) != SAS_OK) return leave(r);
+    if ((r = sas_fwd(p, d.q, d.k, d.v, d.s, d.idx, d.lse_s, d.o, d.lse_o, stream)) != SAS_OK) return leave(r);
     if ((r = sas_bwd(p, d.q, d.k, d.v, d.o, d.dO, d.s, d.idx, d.lse_s, d.lse_o, d.dq, d.dk, d.dv, d.ds, d.ws,
                      d.ws_bytes, stream)) != SAS_OK)
-      return r;
-    if ((e = cudaEventRecord(cr.done[k], cs)) != cudaSuccess) return SAS_ERR_CUDA;
+      return leave(r);
+    if ((e = cudaEventRecord(cr.done[k], cs)) != cudaSuccess) return leave(SAS_ERR_CUDA);
     // outputs back to the host
     if ((e = cudaStreamWaitEvent(cr.down, cr.done[k], 0)) != cudaSuccess ||
         (e = cudaMemcpyAsync(h.o, d.o, b_q, D2H, cr.down)) != cudaSuccess ||
@@ -112,10 +122,8 @@ extern "C" sas_status sas_train_steps_host(const sas_params* p, int n_steps, con
         (e = cudaMemcpyAsync(h.dv, d.dv, b_kv, D2H, cr.down)) != cudaSuccess ||
         (h.ds != nullptr && (e = cudaMemcpyAsync(h.ds, d.ds, b_s, D2H, cr.down)) != cudaSuccess) ||
         (e = cudaEventRecord(cr.out[k], cr.down)) != cudaSuccess)
-      return SAS_ERR_CUDA;
+      return leave(SAS_ERR_CUDA);
   }
   // the caller's stream completes only after the last downloads
-  if (cudaStreamWaitEvent(cs, cr.out[(n_steps - 1) & 1], 0) != cudaSuccess) return SAS_ERR_CUDA;
-  if (n_steps > 1 && cudaStreamWaitEvent(cs, cr.out[n_steps & 1], 0) != cudaSuccess) return SAS_ERR_CUDA;
-  return SAS_OK;
+  return leave(SAS_OK);
 }
