@@ -443,6 +443,31 @@ def run_gpu(args, rank, world, local_rank):
         del step_graph, g_sel, g_split, g_comb
         if sas.sas_get_device_error(stream) != 0:
             raise RuntimeError("device error during decode")
+        # the captured step at other split counts, for the choice of the default (the headline stays
+        # at n_split above); each is the same graph replay with the L2 flushed before it
+        sweep = {}
+        try:
+            for ns in (1, 2, 3, 5, 9):
+                if ns == n_split or (wd.top_k + ns) // ns > 64:
+                    continue
+                o_ns = sas.empty_decode_outputs(pd, ns, device=dev)
+                g_ns = sas.DecodeGraph(pd, xd["q"], xd["k"], xd["v"], xd["cache_len"], xd["s"], ns, o_ns,
+                                       stream=stream)
+                evs = []
+                with torch.cuda.stream(stream):
+                    for i in range(3 + max(10, args.steps)):
+                        torch.sum(flush, dim=0, out=flush_sink)
+                        ev = replay_timed(g_ns.graph)
+                        if i >= 3:
+                            evs.append(ev)
+                torch.cuda.synchronize()
+                sweep[str(ns)] = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+                del g_ns, o_ns
+            if sas.sas_get_device_error(stream) != 0:
+                raise RuntimeError("device error in the split-count sweep")
+        except Exception as e:  # diagnostic only: reported, not raised
+            sweep["error"] = f"{type(e).__name__}: {e}"[:300]
+        line["decode"]["n_split_sweep_ms_per_step"] = sweep
 
     # ---------------- the 128K forward and the budget x length sweep ----------------
     if args.only in ("all", "sweep"):
