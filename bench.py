@@ -547,9 +547,20 @@ def sweep_section(args, sas, stream, dev, pk, dist, world):
         torch.cuda.synchronize()
         out = sas.empty_prefill_outputs(p, device=dev, backward=w.backward)
 
-        def run():
-            sas.prefill_step(p, x["q"], x["k"], x["v"], x["s"], x.get("do"), out, backward=w.backward,
-                             stream=stream)
+        def run(evs=None):
+            # select + LSE, forward, backward; with evs, an event after each call
+            sas.sas_topk_select(p, x["s"], out["idx"], out["lse_s"], stream=stream)
+            if evs is not None:
+                evs[0].record(stream)
+            sas.sas_fwd(p, x["q"], x["k"], x["v"], x["s"], out["idx"], out["lse_s"], out["o"], out["lse_o"],
+                        stream=stream)
+            if evs is not None:
+                evs[1].record(stream)
+            if w.backward:
+                sas.sas_bwd(p, x["q"], x["k"], x["v"], out["o"], x["do"], x["s"], out["idx"], out["lse_s"],
+                            out["lse_o"], out["dq"], out["dk"], out["dv"], out["ds"], out["ws"], stream=stream)
+            if evs is not None:
+                evs[2].record(stream)
 
         n = max(5, min(args.steps, 10))
         with torch.cuda.stream(stream):
@@ -559,12 +570,17 @@ def sweep_section(args, sas, stream, dev, pk, dist, world):
         barrier(dist)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
+        marks = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
         a.record(stream)
         with torch.cuda.stream(stream):
-            for _ in range(n):
-                run()
+            for i in range(n):
+                run(marks[i])
         b.record(stream)
         torch.cuda.synchronize()
+        starts = [a] + [m[2] for m in marks[:-1]]
+        split_ms = {"select": statistics.mean(st.elapsed_time(m[0]) for st, m in zip(starts, marks)),
+                    "fwd": statistics.mean(m[0].elapsed_time(m[1]) for m in marks),
+                    "bwd": statistics.mean(m[1].elapsed_time(m[2]) for m in marks) if w.backward else 0.0}
         if sas.sas_get_device_error(stream) != 0:
             raise RuntimeError(f"device error in {name}")
         ms = max_over_ranks(dist, a.elapsed_time(b), dev) / n
@@ -573,7 +589,10 @@ def sweep_section(args, sas, stream, dev, pk, dist, world):
         tf = job_rate(flops, world, ms * 1e-3) / 1e12
         points.append({"workload": name, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "seq_len": w.seq_len,
                        "top_k": w.top_k, "pass": "fwd+bwd" if w.backward else "fwd", "tflop_per_step": flops / 1e12,
-                       "ms_per_step": ms, "tflops": tf, "frac": tf / (pk["bf16_sustained"] * world)})
+                       "ms_per_step": ms, "tflops": tf, "frac": tf / (pk["bf16_sustained"] * world),
+                       "breakdown_ms": split_ms,
+                       "fwd_tflops": F / (split_ms["fwd"] * 1e-3) / 1e12,
+                       "bwd_tflops": 2.5 * F / (split_ms["bwd"] * 1e-3) / 1e12 if w.backward else None})
         del x, out
         torch.cuda.empty_cache()
     return {"points": points, "peak": pk["bf16_sustained"], "peak_source": pk["source"] + " sustained bf16",
