@@ -34,6 +34,8 @@
 // where one CTA or warp per row would walk the row 32 times.
 #include <cooperative_groups.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace cg = cooperative_groups;
@@ -429,20 +431,20 @@ int scored_cluster_size(int rows, int NB, int sms) {
   return (hist + C - 1) / C > ssc::kMaxSlice ? 0 : C;
 }
 
-// SM count of the current device, fetched once per device (a benign race:
-// every writer stores the same value).
+// SM count of the current device, fetched once per device. Threads that race
+// on the first fetch all store the same value.
 static cudaError_t device_sm_count(int* out) {
-  static int sm_count[64];
+  static std::atomic<int> sm_count[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (sm_count[dev] == 0) {
-    int n = 0;
+  int n = sm_count[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    sm_count[dev] = n;
+    sm_count[dev].store(n, std::memory_order_relaxed);
   }
-  *out = sm_count[dev];
+  *out = n;
   return cudaSuccess;
 }
 
