@@ -83,7 +83,14 @@ typedef enum {
    * log g_m = log σ(s_m): */
   SAS_GATE_LOG_SIGMOID = 2,
   /* log g_m = s_m: */
-  SAS_GATE_LOGIT = 3
+  SAS_GATE_LOGIT = 3,
+  /* The gate outside the softmax (SAS summary §무엇과 다른가, contrasted with
+   * the gate inside): g_m = softmax(s)_m over the history multiplies the
+   * values of block m after a softmax over the plain logits,
+   * o_i = Σ_j g_{m(j)} p_ij v_j (g = 1 for the current block), with no
+   * renormalisation. lse_o is the log-sum-exp of the plain logits. Needs s and
+   * lse_s, like SAS_GATE_LOG_SOFTMAX, and its ds chain is the same. */
+  SAS_GATE_SOFTMAX_OUTSIDE = 4
 } sas_gate_mode;
 
 typedef struct {
@@ -142,7 +149,7 @@ SAS_API sas_status sas_gate_lse(const sas_params* p, const float* s, const int32
  *   k, v   bf16 [B, Hkv, N, d]
  *   s      fp32 [B, Hkv, NQB, NKB]. Read under every gate mode but SAS_GATE_NONE.
  *   idx    int32 [B, Hkv, NQB, K], as written by sas_topk_select.
- *   lse_s  fp32 [B, Hkv, NQB]. Required under SAS_GATE_LOG_SOFTMAX,
+ *   lse_s  fp32 [B, Hkv, NQB]. Required under SAS_GATE_LOG_SOFTMAX and SAS_GATE_SOFTMAX_OUTSIDE,
  *          ignored (may be NULL) under the other modes.
  *   o      bf16 [B, Hq, N, d]. Output.
  *   lse_o  fp32 [B, Hq, N]. Output, may be NULL. Row log-sum-exp of z,
@@ -168,7 +175,8 @@ SAS_API sas_status sas_bwd_workspace_size(const sas_params* p, size_t* bytes);
  *          log g_m summed over block m's tokens, the rows of query block t and
  *          the G heads,
  *            ds[t, m] = dl[t, m]·[m ∈ I_t] − softmax(s[t, 0:t])_m · Σ_{m'∈I_t} dl[t, m']
- *          under SAS_GATE_LOG_SOFTMAX, dl[t, m]·(1 − σ(s[t, m]))·[m ∈ I_t]
+ *          under SAS_GATE_LOG_SOFTMAX and SAS_GATE_SOFTMAX_OUTSIDE (where
+ *          dl = g·∂/∂g = Σ p·g·dOᵀv over the block), dl[t, m]·(1 − σ(s[t, m]))·[m ∈ I_t]
  *          under SAS_GATE_LOG_SIGMOID and dl[t, m]·[m ∈ I_t] under
  *          SAS_GATE_LOGIT. Zero for m >= t, and zero everywhere under
  *          SAS_GATE_NONE. May be NULL under SAS_GATE_NONE.
@@ -201,7 +209,8 @@ SAS_API sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf1
  *   cache_len  int32 [B], 1 <= L <= Lmax
  *   s          fp32 [B, Hkv, NKB]. Read under every gate mode but SAS_GATE_NONE.
  *   idx        int32 [B, Hkv, K] from sas_topk_select (decode form)
- *   lse_s      fp32 [B, Hkv]. Required under SAS_GATE_LOG_SOFTMAX only.
+ *   lse_s      fp32 [B, Hkv]. Required under SAS_GATE_LOG_SOFTMAX and
+ *              SAS_GATE_SOFTMAX_OUTSIDE only.
  *   n_split    1..K+1, with ceil((K+1) / n_split) <= 64 (SAS_ERR_UNSUPPORTED
  *              otherwise): a split covers at most 64 blocks.
  *   o_part     fp32 [B, Hq, n_split, d]. Output.

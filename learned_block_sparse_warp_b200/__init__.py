@@ -21,7 +21,8 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "SAS_GATE_LOG_SOFTMAX", "SAS_GATE_NONE", "SAS_GATE_LOG_SIGMOID", "SAS_GATE_LOGIT", "SasError", "Params", "lib",
+    "SAS_GATE_LOG_SOFTMAX", "SAS_GATE_NONE", "SAS_GATE_LOG_SIGMOID", "SAS_GATE_LOGIT",
+    "SAS_GATE_SOFTMAX_OUTSIDE", "SasError", "Params", "lib",
     "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd", "sas_decode",
     "sas_decode_combine", "sas_decode_paged", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string",
     "sas_version",
@@ -35,6 +36,7 @@ SAS_GATE_LOG_SOFTMAX = 0
 SAS_GATE_NONE = 1
 SAS_GATE_LOG_SIGMOID = 2  # ablation: log g = log σ(s)
 SAS_GATE_LOGIT = 3  # ablation: log g = s
+SAS_GATE_SOFTMAX_OUTSIDE = 4  # ablation: g = softmax(s) weights the values after the softmax
 STATUS = {0: "SAS_OK", 1: "SAS_ERR_INVALID_ARG", 2: "SAS_ERR_UNSUPPORTED", 3: "SAS_ERR_WORKSPACE",
           4: "SAS_ERR_CUDA", 5: "SAS_ERR_TIMEOUT", 6: "SAS_ERR_DEVICE_INDEX"}
 BLOCK = 64

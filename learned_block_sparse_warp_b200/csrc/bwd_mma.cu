@@ -297,6 +297,11 @@ __global__ void __launch_bounds__(256, 1) bwd_main_kernel(
       lam2 = gate_lam2(sh.gate, s[row * sh.NB + j], lse_s != nullptr ? lse_s[row] : 0.f);
     }
     const uint32_t cQ = sQ + stage * TILE, cdO = sdO + stage * TILE;
+    // Gate inside the softmax: log2 g biases the logits. Outside: the logits are
+    // plain, v carries the weight g·p, so dV takes g·p, dZ = p·(g·dP − D), and
+    // dl = Σ p·g·dP (= g ∂/∂g).
+    const float zb = sh.outside ? 0.f : lam2;
+    const float gw = sh.outside ? exp2f(lam2) : 1.f;
 
     // S = Q Kᵀ and dP = dO Vᵀ for rows 16wm.., columns 32wn..
     float sacc[4][4], pacc[4][4];
@@ -336,11 +341,12 @@ __global__ void __launch_bounds__(256, 1) bwd_main_kernel(
           const int cc = col + (c & 1);
           const float Lr = (c >> 1) ? L1 : L0;
           const float Dr = (c >> 1) ? D1 : D0;
-          float pv = exp2f(fmaf(sacc[i][c], sc2, lam2) - Lr);
+          float pv = exp2f(fmaf(sacc[i][c], sc2, zb) - Lr);
           if (diag && cc > row) pv = 0.f;
-          p[c] = pv;
-          z[c] = pv * (pacc[i][c] - Dr);
-          dl_part += z[c];
+          const float gdp = gw * pacc[i][c];
+          p[c] = pv * gw;
+          z[c] = pv * (gdp - Dr);
+          dl_part += sh.outside ? pv * gdp : z[c];
         }
         st_shared_b32(sP + swz<8>(ra, col >> 3) + (col & 7) * 2, pack_bf16x2(p[0], p[1]));
         st_shared_b32(sP + swz<8>(ra + 8, col >> 3) + (col & 7) * 2, pack_bf16x2(p[2], p[3]));
@@ -460,7 +466,7 @@ __global__ void __launch_bounds__(256) bwd_ds_chain_kernel(const float* __restri
   const int32_t* ir = idx + size_t(r) * K;
   const float* dlr = dl + size_t(r) * K;
   const float* sr = s + size_t(r) * NB;
-  if (gate == SAS_GATE_LOG_SOFTMAX) {  // every history block couples through LSE(s)
+  if (gate == SAS_GATE_LOG_SOFTMAX || gate == SAS_GATE_SOFTMAX_OUTSIDE) {  // every history block couples through LSE(s)
     float sum = 0.f;
     for (int kk = lane; kk < n; kk += 32) {
       const int m = ir[kk];

@@ -145,6 +145,10 @@ struct EntryRing {
 // bp and bz are per TMEM buffer because the S and dP issuers wait two steps
 // back; with one barrier they could fall two phases behind. Every other
 // waiter's next phase needs the waiter's own next action first.
+// kOut: the gate weights the values after a softmax over the plain logits
+// (SAS_GATE_SOFTMAX_OUTSIDE): dVᵀ takes g·P, dZ = P·(g·dP − D) and
+// dl = Σ P·g·dP (= g ∂/∂g) instead of Σ dZ.
+template <bool kOut>
 __global__ void __launch_bounds__(bkv::kThreads, 1)
     bwd_kv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ3, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO3,
@@ -368,7 +372,7 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
         float L2 = 0.f;
         asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(L2) : "r"(sL + qs * 512 + row * 4));
         asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(Dr) : "r"(sD + os * 512 + row * 4));
-        L2 = L2 * kLog2e - m.lam2;  // P = exp2(S·sc2 − (L·log2e − λ))
+        L2 = L2 * kLog2e - (kOut ? 0.f : m.lam2);  // P = exp2(S·sc2 − (L·log2e − λ))
         uint32_t vs[16];
         tmem_ld16(tmem + lane_addr + sb * 64 + cg * 16, vs);
         tmem_wait_ld();
@@ -381,13 +385,17 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
         if (i >= 1) ok = mbar_wait(smem_u32(&C.pf), (i - 1) & 1, abort_flag, a.err);
         ok = __all_sync(0xffffffffu, ok);
       }
+      const float gw = kOut ? fast_exp2(m.lam2) : 1.f;  // the gate outside the softmax (1 on the diagonal)
       if (ok) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {  // 16-byte chunk 2 cg + c: 8 kv columns
           const uint32_t off = uint32_t(row * 128 + (((2 * cg + c) ^ (row & 7)) << 4));
+          float w8[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) w8[x] = kOut ? pr[8 * c + x] * gw : pr[8 * c + x];  // dVᵀ's weights
           asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(sP + off),
-                       "r"(pack_bf16x2(pr[8 * c], pr[8 * c + 1])), "r"(pack_bf16x2(pr[8 * c + 2], pr[8 * c + 3])),
-                       "r"(pack_bf16x2(pr[8 * c + 4], pr[8 * c + 5])), "r"(pack_bf16x2(pr[8 * c + 6], pr[8 * c + 7])));
+                       "r"(pack_bf16x2(w8[0], w8[1])), "r"(pack_bf16x2(w8[2], w8[3])),
+                       "r"(pack_bf16x2(w8[4], w8[5])), "r"(pack_bf16x2(w8[6], w8[7])));
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -402,15 +410,28 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
         tmem_ld16(tmem + lane_addr + 128 + sb * 64 + cg * 16, vp);
         tmem_wait_ld();
         float zr[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) zr[x] = pr[x] * (__uint_as_float(vp[x]) - Dr);  // P is 0 where masked
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        if constexpr (kOut) {
 #pragma unroll
-        for (int x = 0; x < 16; x += 4) {
-          s0 += zr[x];
-          s1 += zr[x + 1];
-          s2 += zr[x + 2];
-          s3 += zr[x + 3];
+          for (int x = 0; x < 16; ++x) {
+            const float gdp = gw * __uint_as_float(vp[x]);
+            zr[x] = pr[x] * (gdp - Dr);
+            const float term = pr[x] * gdp;  // dl's term: P·g·dP
+            if ((x & 3) == 0) s0 += term;
+            else if ((x & 3) == 1) s1 += term;
+            else if ((x & 3) == 2) s2 += term;
+            else s3 += term;
+          }
+        } else {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) zr[x] = pr[x] * (__uint_as_float(vp[x]) - Dr);  // P is 0 where masked
+#pragma unroll
+          for (int x = 0; x < 16; x += 4) {
+            s0 += zr[x];
+            s1 += zr[x + 1];
+            s2 += zr[x + 2];
+            s3 += zr[x + 3];
+          }
         }
         dl_part += (s0 + s1) + (s2 + s3);
         // dKᵀ of step i - 1 has read the dZ buffer
@@ -510,7 +531,9 @@ constexpr int kSmem = kStages * kStage + 1024;
 // S = Q Kᵀ and dP = dO Vᵀ (TS MMAs), so shared memory only carries the
 // gathered K and V blocks, six deep. S and dP of consecutive blocks alternate
 // between two TMEM buffers, so the tensor cores compute block i + 1 while the
-// softmax-gradient warps work on block i.
+// softmax-gradient warps work on block i. kOut as in the KV pass: dZ = P·(g·dP − D)
+// over the plain logits.
+template <bool kOut>
 __global__ void __launch_bounds__(bq::kThreads, 1)
     bwd_q_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const uint16_t* __restrict__ q, const uint16_t* __restrict__ dO, BwdSm100Args a) {
@@ -699,7 +722,8 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
       }
       tc_fence_after();
       const uint32_t tS = tmem + lane_addr + sb * 64 + cg * 16, tP = tmem + lane_addr + 128 + sb * 64 + cg * 16;
-      const float off2 = L2 - lam_s[i];
+      const float off2 = kOut ? L2 : L2 - lam_s[i];
+      const float gw = kOut ? fast_exp2(lam_s[i]) : 1.f;  // the gate outside the softmax (1 on the diagonal)
       uint32_t vs[16], vp[16], dz[8];
       tmem_ld16(tS, vs);
       tmem_ld16(tP, vp);
@@ -708,13 +732,15 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
       if (valid && i > 0) {  // every column counts
 #pragma unroll
         for (int x = 0; x < 16; ++x)
-          zr[x] = fast_exp2(fmaf(__uint_as_float(vs[x]), sc2, -off2)) * (__uint_as_float(vp[x]) - Dr);
+          zr[x] = fast_exp2(fmaf(__uint_as_float(vs[x]), sc2, -off2)) *
+                  (kOut ? fmaf(gw, __uint_as_float(vp[x]), -Dr) : __uint_as_float(vp[x]) - Dr);
       } else {
         // none for a missing head, the causal prefix on the diagonal block
         const int n_ok = valid ? min(16, max(0, qpos + 1 - cg * 16)) : 0;
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          const float z = fast_exp2(fmaf(__uint_as_float(vs[x]), sc2, -off2)) * (__uint_as_float(vp[x]) - Dr);
+          const float z = fast_exp2(fmaf(__uint_as_float(vs[x]), sc2, -off2)) *
+                          (kOut ? fmaf(gw, __uint_as_float(vp[x]), -Dr) : __uint_as_float(vp[x]) - Dr);
           zr[x] = x < n_ok ? z : 0.f;
         }
       }
@@ -801,15 +827,15 @@ cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const ui
   a.n_tp = (sh.G + 3) / 4;
   a.scale = sh.scale;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(bwd_kv_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bkv::kSmem)) !=
-      cudaSuccess)
+  auto kv = sh.outside ? bwd_kv_sm100_kernel<true> : bwd_kv_sm100_kernel<false>;
+  auto qk = sh.outside ? bwd_q_sm100_kernel<true> : bwd_q_sm100_kernel<false>;
+  if ((e = cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, bkv::kSmem)) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(bwd_q_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bq::kSmem)) !=
-      cudaSuccess)
+  if ((e = cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, bq::kSmem)) != cudaSuccess)
     return e;
-  bwd_kv_sm100_kernel<<<dim3(sh.NB, sh.Hkv, sh.B), bkv::kThreads, bkv::kSmem, st>>>(tq3, tk, tv, tdo3, tl, td, a);
+  kv<<<dim3(sh.NB, sh.Hkv, sh.B), bkv::kThreads, bkv::kSmem, st>>>(tq3, tk, tv, tdo3, tl, td, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_q_sm100_kernel<<<dim3(sh.NB, sh.Hkv * a.n_hp, sh.B), bq::kThreads, bq::kSmem, st>>>(tk, tv, q, dO, a);
+  qk<<<dim3(sh.NB, sh.Hkv * a.n_hp, sh.B), bq::kThreads, bq::kSmem, st>>>(tk, tv, q, dO, a);
   return cudaGetLastError();
 }
 

@@ -23,14 +23,17 @@ struct Shape {
   int B, Hq, Hkv, G, d, N, NB, K;
   float scale;  // softmax scale (1/sqrt(d) unless given)
   int gate;     // sas_gate_mode
-  int gated;    // 1 when the gate puts a log g inside the softmax (every mode but SAS_GATE_NONE)
+  int gated;    // 1 when a gate applies (every mode but SAS_GATE_NONE)
+  int outside;  // 1 when the gate weights the values after the softmax (SAS_GATE_SOFTMAX_OUTSIDE)
 };
 
 // λ_m of a selected history block in log2 units, log g_m · log2 e, for the gate
-// mode: s_m − LSE(s) (softmax-normalised), log σ(s_m), s_m (raw logit), or 0.
+// mode: s_m − LSE(s) (softmax-normalised, inside or outside the softmax),
+// log σ(s_m), s_m (raw logit), or 0.
 __device__ __forceinline__ float gate_lam2(int gate, float s_m, float lse) {
   switch (gate) {
-    case SAS_GATE_LOG_SOFTMAX: return (s_m - lse) * kLog2e;
+    case SAS_GATE_LOG_SOFTMAX:
+    case SAS_GATE_SOFTMAX_OUTSIDE: return (s_m - lse) * kLog2e;
     case SAS_GATE_LOG_SIGMOID: return (fminf(s_m, 0.f) - log1pf(expf(-fabsf(s_m)))) * kLog2e;
     case SAS_GATE_LOGIT: return s_m * kLog2e;
     default: return 0.f;

@@ -51,7 +51,7 @@ struct DecodeArgs {
   float* o_part;
   float* lse_part;
   int* err;
-  int B, Hkv, Lmax, K, gate, gated, n_split, per_max, items_per_chunk;
+  int B, Hkv, Lmax, K, gate, gated, outside, n_split, per_max, items_per_chunk;
   float scale;
 };
 
@@ -220,7 +220,9 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       __syncthreads();
       const uint32_t st = ring + (task % STAGES) * STAGEB;
       const int ntok = t_ntok[task];
-      const float lam2 = t_lam[task];
+      // the gate inside the softmax biases the logits by log2 g; outside, it weights P·V by g
+      const float lam2 = a.outside ? 0.f : t_lam[task];
+      const float gw = a.outside ? exp2f(t_lam[task]) : 1.f;
       const int flags = t_flags[task];
       if (flags & 1) {
 #pragma unroll
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       for (int n = 0; n < 2; ++n) {
         const int tok = 16 * warp + 8 * n + 2 * (lane & 3);
         const uint32_t addr = sP + swz<8>(g_row, tok >> 3) + (tok & 7) * 2;
-        asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(addr), "r"(pack_bf16x2(pv[2 * n], pv[2 * n + 1])));
+        asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(addr), "r"(pack_bf16x2(pv[2 * n] * gw, pv[2 * n + 1] * gw)));
       }
 #pragma unroll
       for (int j = 0; j < DW / 8; ++j) {
@@ -429,6 +431,7 @@ static cudaError_t launch_decode_d(const Shape& sh, const uint16_t* q, const uin
   a.K = sh.K;
   a.gate = sh.gate;
   a.gated = sh.gated;
+  a.outside = sh.outside;
   a.n_split = n_split;
   a.per_max = (sh.K + 1 + n_split - 1) / n_split;
   a.items_per_chunk = max(1, min(dec::kThreads, dec::kMaxTasks / a.per_max));

@@ -100,8 +100,10 @@ __global__ void __launch_bounds__(128) fwd_mma_kernel(const uint16_t* __restrict
         mma_bf16_16816(sacc[2 * np + 1], a, b2, b3);
       }
     }
-    // gated logits in the log2 domain; causal mask on the current block
-    const float lam2 = lam_s[i];
+    // gated logits in the log2 domain; causal mask on the current block. The gate
+    // outside the softmax leaves the logits plain and weights P·V by g instead.
+    const float lam2 = sh.outside ? 0.f : lam_s[i];
+    const float gw = sh.outside ? exp2f(lam_s[i]) : 1.f;
     const bool diag = (i == 0);
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -148,10 +150,10 @@ __global__ void __launch_bounds__(128) fwd_mma_kernel(const uint16_t* __restrict
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t a[4];
-      a[0] = pack_bf16x2(sacc[2 * kk][0], sacc[2 * kk][1]);
-      a[1] = pack_bf16x2(sacc[2 * kk][2], sacc[2 * kk][3]);
-      a[2] = pack_bf16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
-      a[3] = pack_bf16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
+      a[0] = pack_bf16x2(sacc[2 * kk][0] * gw, sacc[2 * kk][1] * gw);
+      a[1] = pack_bf16x2(sacc[2 * kk][2] * gw, sacc[2 * kk][3] * gw);
+      a[2] = pack_bf16x2(sacc[2 * kk + 1][0] * gw, sacc[2 * kk + 1][1] * gw);
+      a[3] = pack_bf16x2(sacc[2 * kk + 1][2] * gw, sacc[2 * kk + 1][3] * gw);
 #pragma unroll
       for (int dp = 0; dp < D / 16; ++dp) {
         uint32_t b0, b1, b2, b3;

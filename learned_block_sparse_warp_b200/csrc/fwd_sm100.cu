@@ -52,6 +52,9 @@ struct FwdSm100Args {
   float scale;
 };
 
+// kOut: the gate weights the values after a softmax over the plain logits
+// (SAS_GATE_SOFTMAX_OUTSIDE) instead of entering the logits as log g.
+template <bool kOut>
 __global__ void __launch_bounds__(fsm::kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, FwdSm100Args a) {
@@ -207,7 +210,8 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       }
       tc_fence_after();
       const int nb = min(2, nl - 2 * p);
-      const float lamA = lam_s[2 * p], lamB = nb > 1 ? lam_s[2 * p + 1] : 0.f;
+      // log2 g of the pair's two blocks, as a logit bias (the gate outside the softmax adds none)
+      const float lamA = kOut ? 0.f : lam_s[2 * p], lamB = (kOut || nb < 2) ? 0.f : lam_s[2 * p + 1];
       const bool diag = (p == 0);  // block A of pair 0 is the causal current block
       // The pair's S row (up to 128 columns) comes out of TMEM in four loads and
       // one wait, and stays in registers. Raw row max per 64-column block; the
@@ -271,6 +275,9 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         const float off = (ch2 == 0 ? lamA : lamB) - m_used;  // p = 2^(S·sc2 + λ − m)
         uint32_t pk[32];
         float s0 = 0.f, s1 = 0.f;
+        // gate outside: the row sum takes p, the values take g·p
+        __nv_bfloat162 gw2;
+        if constexpr (kOut) gw2 = __float2bfloat162_rn(fast_exp2(lam_s[2 * p + ch2]));
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const float p0 = fast_exp2(fmaf(__uint_as_float(v[64 * ch2 + 2 * e]), sc2, off));
@@ -278,6 +285,10 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
           s0 += p0;
           s1 += p1;
           pk[e] = pack_bf16x2(p0, p1);
+          if constexpr (kOut) {  // g·p in bf16: p and g rounded once each, then their product
+            __nv_bfloat162 pg = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&pk[e]), gw2);
+            pk[e] = *reinterpret_cast<uint32_t*>(&pg);
+          }
         }
         l += s0 + s1;
         tmem_st32(tS + ch2 * 32, pk);  // P columns [32 ch2, 32 ch2 + 32)
@@ -413,8 +424,8 @@ cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t*
   if (!make_tmap_bf16_2d(&tq, q, rq, 128) || !make_tmap_bf16_2d(&tk, k, rkv, 128) ||
       !make_tmap_bf16_2d(&tv, v, rkv, 128))
     return cudaErrorInvalidValue;
-  cudaError_t e =
-      cudaFuncSetAttribute(fwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fsm::kSmemBytes);
+  auto kern = sh.outside ? fwd_sm100_kernel<true> : fwd_sm100_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fsm::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdSm100Args a;
   a.idx = idx;
@@ -435,7 +446,7 @@ cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t*
   a.n_tp = (sh.G + 3) / 4;
   a.scale = sh.scale;
   dim3 grid(sh.NB, sh.Hkv * a.n_tp, sh.B);
-  fwd_sm100_kernel<<<grid, fsm::kThreads, fsm::kSmemBytes, st>>>(tq, tk, tv, a);
+  kern<<<grid, fsm::kThreads, fsm::kSmemBytes, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

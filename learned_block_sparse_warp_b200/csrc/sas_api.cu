@@ -65,11 +65,12 @@ bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 
 // Gate inputs: s for every gate mode but SAS_GATE_NONE, and lse_s for the
-// softmax-normalised gate. The ablation modes do not read lse_s (it may be NULL).
+// softmax-normalised gate, inside or outside the softmax. The activation
+// ablations do not read lse_s (it may be NULL).
 bool gate_inputs_ok(const Shape& sh, const float* s, const float* lse_s) {
   if (!sh.gated) return true;
   if (!ok_ptr(s) || !ok_opt(lse_s)) return false;
-  return sh.gate != SAS_GATE_LOG_SOFTMAX || lse_s != nullptr;
+  return (sh.gate != SAS_GATE_LOG_SOFTMAX && sh.gate != SAS_GATE_SOFTMAX_OUTSIDE) || lse_s != nullptr;
 }
 
 // Checks the shared parameters and fills the kernel-side shape.
@@ -78,7 +79,7 @@ sas_status make_shape(const sas_params* p, Shape* sh) {
   if (p->batch < 1 || p->n_q_heads < 1 || p->n_kv_heads < 1 || p->seq_len < 1 || p->top_k < 1)
     return SAS_ERR_INVALID_ARG;
   if (p->n_q_heads % p->n_kv_heads != 0) return SAS_ERR_INVALID_ARG;
-  if (p->gate_mode < SAS_GATE_LOG_SOFTMAX || p->gate_mode > SAS_GATE_LOGIT) return SAS_ERR_INVALID_ARG;
+  if (p->gate_mode < SAS_GATE_LOG_SOFTMAX || p->gate_mode > SAS_GATE_SOFTMAX_OUTSIDE) return SAS_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.f) || isinf(p->softmax_scale)) return SAS_ERR_INVALID_ARG;
   if (p->top_k > sas::kMaxTopK) return SAS_ERR_INVALID_ARG;
   static_assert(sas::kMaxTopK <= (1 << sas::kSlotBits), "reverse-index slot field");
@@ -102,6 +103,7 @@ sas_status make_shape(const sas_params* p, Shape* sh) {
   sh->scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(float(p->head_dim));
   sh->gate = p->gate_mode;
   sh->gated = p->gate_mode != SAS_GATE_NONE ? 1 : 0;
+  sh->outside = p->gate_mode == SAS_GATE_SOFTMAX_OUTSIDE ? 1 : 0;
   return SAS_OK;
 }
 

@@ -162,7 +162,10 @@ def test_gate_ablation_inputs_checked():
     for mode in (2, 3):
         assert _fwd(_p(gate_mode=mode), s=None) == INVALID
     assert _fwd(_p(gate_mode=0), lse_s=None) == INVALID
-    assert _fwd(_p(gate_mode=4)) == INVALID
+    # the gate outside the softmax is softmax-normalised: it needs s and lse_s
+    assert _fwd(_p(gate_mode=4), s=None) == INVALID
+    assert _fwd(_p(gate_mode=4), lse_s=None) == INVALID
+    assert _fwd(_p(gate_mode=5)) == INVALID
     c = _p(gate_mode=2).c()
     assert lib.sas_decode(ctypes.byref(c), A, A, A, A, None, A, None, 2, A, A, None) == INVALID  # s missing
 
