@@ -292,7 +292,15 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         l += s0 + s1;
         tmem_st32(tS + ch2 * 32, pk);
       };
+      // the turn guards the exponentials only: it passes as soon as the last block's are done
+      auto pass_turn = [&]() {
+        if (n_tiles == 2) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bar_turn[r ^ 1]));
+        }
+      };
       block_p(0);
+      if (nb == 1) pass_turn();
       if (p > 0 && __any_sync(0xffffffffu, grow)) {
         // O holds PV of earlier pairs, complete because S_r(p) completed after it. It is
         // rescaled before the first block's PV of this pair is released, 16 columns at a time.
@@ -310,13 +318,10 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       mbar_arrive(smem_u32(&bar_p[r]));
       if (nb > 1) {
         block_p(1);
+        pass_turn();
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(smem_u32(&bar_pb[r]));
-      }
-      if (n_tiles == 2) {  // pass the turn to the other tile
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_turn[r ^ 1]));
       }
     }
     if (ok) ok = mbar_wait(smem_u32(&bar_o[r]), (n_pairs - 1) & 1, abort_flag, a.err);
