@@ -66,8 +66,10 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
   // bar_turn[r]: tile r's softmax may run its exponentials. The two tiles take
   // turns, so one tile's exponentials overlap the other tile's MMAs instead of
   // both contending for the SM's exponential units at once.
+  // bar_p[r] / bar_pb[r]: tile r's P of the pair's first / second 64-column block is in TMEM,
+  // so the PV of the first block starts while the second block's exponentials run.
   __shared__ __align__(8) uint64_t bar_q, bar_full[fsm::kStages], bar_empty[fsm::kStages], bar_s[2], bar_p[2],
-      bar_o[2], bar_fin, bar_turn[2];
+      bar_pb[2], bar_o[2], bar_fin, bar_turn[2];
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
 
@@ -100,6 +102,7 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       for (int r = 0; r < 2; ++r) {
         mbar_init(smem_u32(&bar_s[r]), 1);
         mbar_init(smem_u32(&bar_p[r]), 128);
+        mbar_init(smem_u32(&bar_pb[r]), 128);
         mbar_init(smem_u32(&bar_o[r]), 1);
       }
       mbar_init(smem_u32(&bar_fin), n_tiles);
@@ -184,8 +187,14 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         mma_commit(smem_u32(&bar_s[r]));
         if (!(ok = mbar_wait(smem_u32(&bar_p[r]), p & 1, abort_flag, a.err))) break;
         tc_fence_after();
-        for (int jj = 0; jj < 4 * nb; ++jj)
+        for (int jj = 0; jj < 4; ++jj)  // the first block's 64 tokens
           mma_ts(tO, tS + jj * 8, desc_advance(dV0, so + jj * 2048), idPV, (p > 0 || jj > 0) ? 1u : 0u);
+        if (nb > 1) {  // the second block's, once its P is in (every pair but an odd last one)
+          if (!(ok = mbar_wait(smem_u32(&bar_pb[r]), p & 1, abort_flag, a.err))) break;
+          tc_fence_after();
+          for (int jj = 4; jj < 8; ++jj)
+            mma_ts(tO, tS + jj * 8, desc_advance(dV0, so + jj * 2048), idPV, 1u);
+        }
         mma_commit(smem_u32(&bar_o[r]));
         mma_commit(smem_u32(&bar_empty[st]));
       }
@@ -270,8 +279,9 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
           break;
         }
       }
-      // probabilities, row sum, bf16 P over the S columns (all read above)
-      for (int ch2 = 0; ch2 < nb; ++ch2) {
+      // probabilities, row sum, bf16 P over the S columns (all read above), one 64-column
+      // block at a time: block ch2's P goes to TMEM columns [32 ch2, 32 ch2 + 32)
+      auto block_p = [&](const int ch2) {
         const float off = (ch2 == 0 ? lamA : lamB) - m_used;  // p = 2^(S·sc2 + λ − m)
         uint32_t pk[32];
         float s0 = 0.f, s1 = 0.f;
@@ -291,25 +301,38 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
           }
         }
         l += s0 + s1;
-        tmem_st32(tS + ch2 * 32, pk);  // P columns [32 ch2, 32 ch2 + 32)
-      }
+        tmem_st32(tS + ch2 * 32, pk);
+      };
+      // the turn guards the exponentials only: it passes as soon as the last block's are done
+      auto pass_turn = [&]() {
+        if (n_tiles == 2) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bar_turn[r ^ 1]));
+        }
+      };
+      block_p(0);
+      if (nb == 1) pass_turn();
       if (p > 0 && __any_sync(0xffffffffu, grow)) {
-        // O holds PV of earlier pairs, complete because S_r(p) completed after it
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t w[32];
-          tmem_ld32(tO + ch * 32, w);
+        // O holds PV of earlier pairs, complete because S_r(p) completed after it. It is
+        // rescaled before the first block's PV of this pair is released, 16 columns at a time.
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t w[16];
+          tmem_ld16(tO + ch * 16, w);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * alpha);
-          tmem_st32(tO + ch * 32, w);
+          for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * alpha);
+          tmem_st16(tO + ch * 16, w);
         }
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&bar_p[r]));
-      if (n_tiles == 2) {  // pass the turn to the other tile
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_turn[r ^ 1]));
+      if (nb > 1) {
+        block_p(1);
+        pass_turn();
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bar_pb[r]));
       }
     }
     if (ok) ok = mbar_wait(smem_u32(&bar_o[r]), (n_pairs - 1) & 1, abort_flag, a.err);
