@@ -163,8 +163,17 @@ SAS_API sas_status sas_fwd(const sas_params* p, const sas_bf16* q, const sas_bf1
  * inside the softmax, chained through g = softmax(s); sparse scope)
  * ------------------------------------------------------------------------- */
 
-/* Bytes of device workspace that sas_bwd needs for these params. */
+/* Bytes of device workspace for the fastest form of sas_bwd. At head_dim 128
+ * it includes one bf16 dZ tile per (query block, attended block, pair of
+ * query heads): 16 KB × B·Hkv·Σ_t (1 + min(K, t))·ceil(G/2), about 4.3 GB at
+ * B 1, 8 KV heads, G 4, N 32768, K 32. The KV-major pass stores dZ there and
+ * the dQ pass reads it back instead of recomputing S and dP. */
 SAS_API sas_status sas_bwd_workspace_size(const sas_params* p, size_t* bytes);
+
+/* The smallest workspace sas_bwd accepts. With less than
+ * sas_bwd_workspace_size bytes (but at least this many) the dQ pass
+ * recomputes S and dP itself: the same results, more time, no dZ tiles. */
+SAS_API sas_status sas_bwd_workspace_size_min(const sas_params* p, size_t* bytes);
 
 /* Gradients of ⟨dO, o⟩ with the selection idx held fixed.
  *   Inputs: q, k, v, s, idx, lse_s as in sas_fwd. o and lse_o are the
@@ -180,9 +189,10 @@ SAS_API sas_status sas_bwd_workspace_size(const sas_params* p, size_t* bytes);
  *          under SAS_GATE_LOG_SIGMOID and dl[t, m]·[m ∈ I_t] under
  *          SAS_GATE_LOGIT. Zero for m >= t, and zero everywhere under
  *          SAS_GATE_NONE. May be NULL under SAS_GATE_NONE.
- *   ws     device workspace of at least sas_bwd_workspace_size bytes,
- *          256-byte aligned. Its contents on entry do not matter. The call
- *          overwrites it.
+ *   ws     device workspace, 256-byte aligned, of at least
+ *          sas_bwd_workspace_size_min bytes (SAS_ERR_WORKSPACE otherwise).
+ *          With sas_bwd_workspace_size bytes or more the faster form runs.
+ *          Its contents on entry do not matter. The call overwrites it.
  * idx must be in the form sas_topk_select writes: ascending, −1 padded.
  * Other index lists are memory-safe but their gradients are unspecified. */
 SAS_API sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, const sas_bf16* v,
@@ -359,7 +369,8 @@ typedef struct {
 
 /* One set of caller-owned device buffers for a step, with the layouts of the
  * host buffers, plus idx int32 [B, Hkv, NQB, K], lse_s fp32 [B, Hkv, NQB], and
- * the backward workspace (sas_bwd_workspace_size bytes, 256-byte aligned). ds
+ * the backward workspace (at least sas_bwd_workspace_size_min bytes, 256-byte
+ * aligned; sas_bwd_workspace_size bytes select the faster backward). ds
  * is required under every gate mode but SAS_GATE_NONE. */
 typedef struct {
   sas_bf16 *q, *k, *v, *dO, *o, *dq, *dk, *dv;

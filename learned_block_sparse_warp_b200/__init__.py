@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "SAS_GATE_LOG_SOFTMAX", "SAS_GATE_NONE", "SAS_GATE_LOG_SIGMOID", "SAS_GATE_LOGIT",
     "SAS_GATE_SOFTMAX_OUTSIDE", "SasError", "Params", "lib",
-    "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd", "sas_decode",
+    "sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd_workspace_size", "sas_bwd_workspace_size_min", "sas_bwd",
+    "sas_decode",
     "sas_decode_combine", "sas_decode_paged", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string",
     "sas_version",
     "DecodeGraph", "sas_selftest_wait_timeout", "sas_block_mean_keys", "sas_decode_select_scored",
@@ -78,6 +79,7 @@ def _load() -> ctypes.CDLL:
         "sas_gate_lse": [P, vp, vp, vp, vp],
         "sas_fwd": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "sas_bwd_workspace_size": [P, ctypes.POINTER(sz)],
+        "sas_bwd_workspace_size_min": [P, ctypes.POINTER(sz)],
         "sas_bwd": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "sas_decode": [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp],
         "sas_decode_paged": [P, vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp],
@@ -202,6 +204,12 @@ def sas_fwd(p: Params, q, k, v, s, idx, lse_s, o, lse_o=None, stream=None) -> No
 def sas_bwd_workspace_size(p: Params) -> int:
     n = ctypes.c_size_t(0)
     _check("sas_bwd_workspace_size", lib.sas_bwd_workspace_size(ctypes.byref(p.c()), ctypes.byref(n)))
+    return int(n.value)
+
+
+def sas_bwd_workspace_size_min(p: Params) -> int:
+    n = ctypes.c_size_t(0)
+    _check("sas_bwd_workspace_size_min", lib.sas_bwd_workspace_size_min(ctypes.byref(p.c()), ctypes.byref(n)))
     return int(n.value)
 
 

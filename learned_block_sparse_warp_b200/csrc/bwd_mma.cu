@@ -33,22 +33,29 @@
 namespace sas {
 
 struct BwdWs {
-  float* dq_acc;   // [B, Hq, N, d] fp32
+  float* dq_acc;   // [B, Hq, N, d] fp32 (d = 64 path only)
   float* drow;     // [B, Hq, N]
   float* dl;       // [B, Hkv, NB, K]
   int* rev_cnt;    // [B, Hkv, NB]
   int* rev_off;    // [B, Hkv, NB + 1]
   int* rev_list;   // [B, Hkv, NB * K]: (t << kSlotBits) | slot
   float* rev_lam;  // [B, Hkv, NB * K]: log2-domain gate of each reverse-index entry
+  uint16_t* dz;    // d = 128 with spill: [B, Hkv, Σ_t (1 + min(K, t)), ceil(G/2)] tiles of 128 x 64 bf16
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-size_t bwd_ws_layout(const Shape& sh, void* base, BwdWs* ws) {
+long long bwd_dz_tiles(const Shape& sh);
+
+// The stored-dZ backward needs one 16 KB tile per (query block, attended block,
+// head pair); its tile index must fit a TMA coordinate.
+bool bwd_can_spill(const Shape& sh) { return sh.d == 128 && bwd_dz_tiles(sh) < (1LL << 31); }
+
+size_t bwd_ws_layout(const Shape& sh, bool spill, void* base, BwdWs* ws) {
   const size_t bhq = size_t(sh.B) * sh.Hq, bhk = size_t(sh.B) * sh.Hkv;
   size_t off = 0;
   size_t o_dq = off;
-  off = align256(off + bhq * sh.N * sh.d * sizeof(float));
+  if (sh.d != 128) off = align256(off + bhq * sh.N * sh.d * sizeof(float));
   size_t o_dr = off;
   off = align256(off + bhq * sh.N * sizeof(float));
   size_t o_dl = off;
@@ -61,15 +68,18 @@ size_t bwd_ws_layout(const Shape& sh, void* base, BwdWs* ws) {
   off = align256(off + bhk * sh.NB * sh.K * sizeof(int));
   size_t o_lam = off;
   off = align256(off + bhk * sh.NB * sh.K * sizeof(float));
+  size_t o_dz = off;
+  if (spill) off = align256(off + size_t(bwd_dz_tiles(sh)) * 128 * 64 * sizeof(uint16_t));
   if (ws != nullptr) {
     char* p = static_cast<char*>(base);
-    ws->dq_acc = reinterpret_cast<float*>(p + o_dq);
+    ws->dq_acc = sh.d != 128 ? reinterpret_cast<float*>(p + o_dq) : nullptr;
     ws->drow = reinterpret_cast<float*>(p + o_dr);
     ws->dl = reinterpret_cast<float*>(p + o_dl);
     ws->rev_cnt = reinterpret_cast<int*>(p + o_cnt);
     ws->rev_off = reinterpret_cast<int*>(p + o_off);
     ws->rev_list = reinterpret_cast<int*>(p + o_list);
     ws->rev_lam = reinterpret_cast<float*>(p + o_lam);
+    ws->dz = spill ? reinterpret_cast<uint16_t*>(p + o_dz) : nullptr;
   }
   return off;
 }
@@ -494,15 +504,16 @@ __global__ void __launch_bounds__(256) bwd_ds_chain_kernel(const float* __restri
 cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                    const uint16_t* dO, const float* s, const int32_t* idx, const float* lse_s,
                                    const float* lse_o, const float* drow, const int* rev_off, const int* rev_list,
-                                   const float* rev_lam, float* dl, uint16_t* dq, uint16_t* dk, uint16_t* dv, int* err, cudaStream_t st);
+                                   const float* rev_lam, float* dl, uint16_t* dz, uint16_t* dq, uint16_t* dk,
+                                   uint16_t* dv, int* err, cudaStream_t st);
 
 template <int D>
 static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                 const uint16_t* o, const uint16_t* dO, const float* s, const int32_t* idx,
                                 const float* lse_s, const float* lse_o, uint16_t* dq, uint16_t* dk, uint16_t* dv,
-                                float* ds, void* ws_base, int* err, cudaStream_t st) {
+                                float* ds, void* ws_base, bool spill, int* err, cudaStream_t st) {
   BwdWs ws;
-  bwd_ws_layout(sh, ws_base, &ws);
+  bwd_ws_layout(sh, spill, ws_base, &ws);
   const size_t rows_q = size_t(sh.B) * sh.Hq * sh.N;
   const int nbh = sh.B * sh.Hkv;
   cudaError_t e;
@@ -519,10 +530,9 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
   revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
   revidx_fill_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_off, ws.rev_list, s, lse_s,
                                                     sh.gate, D == 128 ? ws.rev_lam : nullptr);
-  if (D == 128) {  // tcgen05 passes: dK/dV/dl KV-major, then dQ query-major; no dQ accumulator
+  if (D == 128) {  // tcgen05 passes: dK/dV/dl (and the dZ tiles) KV-major, then dQ query-major
     if ((e = launch_bwd_passes_sm100(sh, q, k, v, dO, s, idx, lse_s, lse_o, ws.drow, ws.rev_off, ws.rev_list,
-                                     ws.rev_lam, ws.dl,
-                                     dq, dk, dv, err, st)) != cudaSuccess)
+                                     ws.rev_lam, ws.dl, ws.dz, dq, dk, dv, err, st)) != cudaSuccess)
       return e;
     if (ds != nullptr) {
       const int rows = nbh * sh.NB;
@@ -550,9 +560,10 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
 cudaError_t launch_bwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                            const uint16_t* o, const uint16_t* dO, const float* s, const int32_t* idx,
                            const float* lse_s, const float* lse_o, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* ds,
-                           void* ws, int* err, cudaStream_t st) {
-  if (sh.d == 128) return launch_bwd_d<128>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, err, st);
-  return launch_bwd_d<64>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, err, st);
+                           void* ws, bool spill, int* err, cudaStream_t st) {
+  if (sh.d == 128)
+    return launch_bwd_d<128>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, spill, err, st);
+  return launch_bwd_d<64>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, false, err, st);
 }
 
 }  // namespace sas

@@ -44,7 +44,17 @@ struct BwdSm100Args {
   int* err;
   int B, Hq, Hkv, G, N, NB, K, gate, gated, n_hp, n_tp;
   float scale;
+  int spill;            // 1: the KV pass stores every dZ tile and the dQ pass reads them back
+  long long dz_slots;   // dZ slots per (batch, KV head): Σ_t (1 + min(K, t))
 };
+
+// First dZ slot of query block t: Σ_{t' < t} (1 + min(K, t')). Slot 0 of a query
+// block holds its diagonal block, slot 1 + s the block in idx[t][s].
+__host__ __device__ __forceinline__ long long dz_slot_base(int t, int K) {
+  const long long tt = t, kk = K;
+  if (tt <= kk + 1) return tt + tt * (tt - 1) / 2;
+  return (kk + 1) + kk * (kk + 1) / 2 + (tt - kk - 1) * (kk + 1);
+}
 
 // ===========================================================================
 // Pass 1: dK, dV and dl, KV-major
@@ -142,6 +152,7 @@ struct EntryRing {
 //                waits bd[b] and zf (step i - 1), writes dZ -> bz[b]
 //   dVᵀ          waits fo[o], bp[b]                          -> pf, eo[o]
 //   dKᵀ          waits fq[q], bz[b]                          -> zf, eq[q]
+//                and, when spilling, stores the dZ tile     -> zf (second arrival, once it is read)
 // bp and bz are per TMEM buffer because the S and dP issuers wait two steps
 // back; with one barrier they could fall two phases behind. Every other
 // waiter's next phase needs the waiter's own next action first.
@@ -153,7 +164,7 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
     bwd_kv_sm100_kernel(const __grid_constant__ CUtensorMap tmQ3, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO3,
                         const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmD,
-                        BwdSm100Args a) {
+                        const __grid_constant__ CUtensorMap tmDZ, BwdSm100Args a) {
   using namespace sm100;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
@@ -203,7 +214,7 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
         mbar_init(smem_u32(&C.bz[r]), bkv::kSoftWarps);
       }
       mbar_init(smem_u32(&C.pf), 1);
-      mbar_init(smem_u32(&C.zf), 1);
+      mbar_init(smem_u32(&C.zf), a.spill ? 2 : 1);  // dKᵀ's commit, and the dZ store's read when spilling
       mbar_init(smem_u32(&C.fin), 2);
       fence_barrier_init();
     }
@@ -327,14 +338,28 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
         if (!(ok = mbar_wait(smem_u32(is_v ? &C.fo[st] : &C.fq[st]), use & 1, abort_flag, a.err))) break;
         if (!(ok = mbar_wait(smem_u32(is_v ? &C.bp[sb] : &C.bz[sb]), (i >> 1) & 1, abort_flag, a.err))) break;
         tc_fence_after();
+        // read before the MMAs: their commit on eq lets the producer refill this Q slot and its meta
+        const bkv::Meta m = is_v ? bkv::Meta{0, 0, 0, 0.f} : C.meta[st];
         const uint32_t so = st * bkv::kTile;
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           mma_ss(tG, desc_advance(dGa, so + k * 2048), desc_advance(dGb, k * 2048), idG, (i > 0 || k > 0) ? 1u : 0u);
         mma_commit(smem_u32(is_v ? &C.pf : &C.zf));
         mma_commit(smem_u32(is_v ? &C.eo[st] : &C.eq[st]));
+        if (!is_v && a.spill) {
+          // The dZ tile also goes to the workspace, where the dQ pass reads it back
+          // instead of recomputing S and dP. The buffer is released (the second
+          // arrival on zf) once the store has read it.
+          const long long tile =
+              (static_cast<long long>(bh) * a.dz_slots + dz_slot_base(m.t, a.K) + (m.slot + 1)) * a.n_hp + (i % a.n_hp);
+          tma_store_3d(&tmDZ, 0, 0, int(tile), sZ);
+          bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(smem_u32(&C.zf));
+        }
       }
       mma_commit(smem_u32(&C.fin));
+      if (!is_v && a.spill) bulk_wait_all();
     }
   } else if (warp >= 4 && warp < 4 + bkv::kSoftWarps) {
     // ------------------------------------------------------------ softmax gradient
@@ -786,19 +811,208 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
   }
 }
 
+// ===========================================================================
+// Pass 2 with stored dZ: dQ = scale · Σ_j dZ_tj K_j, query-major
+// ===========================================================================
+namespace bdq {
+constexpr int kThreads = 192;          // 0 TMA, 1 TMEM + MMA issue, 2-5 epilogue
+constexpr int kTileZ = 128 * 64 * 2;   // one stored dZ tile: 128 rows (a head pair) x 64 kv bf16
+constexpr int kHalfK = 64 * 128;       // one d-half of a 64-row K block
+constexpr int kStage = 2 * kHalfK + 2 * kTileZ;  // K block + up to two dZ tiles: 48 KB
+constexpr int kStages = 2;             // two CTAs per SM: one's start and end hide under the other's loop
+constexpr int kSmem = kStages * kStage + 1024;
+}  // namespace bdq
+
+// One CTA per (batch, KV head, query block, up to two head pairs). The list of
+// the block's dZ slots is [diagonal, idx[t][0], idx[t][1], ...]. For each,
+// the producer brings the K block and the stored dZ tiles of the CTA's head
+// pairs into a stage, and one thread issues dQ_r += dZ_r · K as four M = 128,
+// N = 128, K = 16 MMAs per tile (dZ K-major, K MN-major), accumulating in TMEM.
+// No exponential and no recomputed product: the KV pass derived dZ already.
+__global__ void __launch_bounds__(bdq::kThreads, 2)
+    bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmDZ,
+                        BwdSm100Args a) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int list_s[kMaxTopK + 1];  // (m << kSlotBits) | dZ slot
+  __shared__ int nlist_s;
+  __shared__ __align__(8) uint64_t bar_full[bdq::kStages], bar_empty[bdq::kStages], bar_fin;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int t = a.NB - 1 - int(blockIdx.x);
+  const int n_pp = (a.n_hp + 1) / 2;  // CTAs per KV head
+  const int h = int(blockIdx.y) / n_pp, pp = int(blockIdx.y) % n_pp;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hp0 = 2 * pp;
+  const int n_tiles = min(2, a.n_hp - hp0);
+  const size_t bh = size_t(b) * a.Hkv + h;
+  const long long slot0 = static_cast<long long>(bh) * a.dz_slots + dz_slot_base(t, a.K);
+  volatile int* abort_flag = &abort_s;
+
+  if (threadIdx.x == 0) abort_s = 0;
+  if (warp == 0) {
+    // list: the diagonal (slot 0), then every valid idx entry s (slot s + 1); an entry
+    // outside the history is skipped and raised, the first -1 ends the list
+    const int n = min(a.K, t);
+    const int32_t* row = a.idx + (bh * a.NB + t) * size_t(a.K);
+    int cnt = 0;
+    bool stop = false;
+    for (int base = 0; base < n && !stop; base += 32) {
+      const int k = base + lane;
+      const int m = k < n ? row[k] : -1;
+      const bool end = k < n && m < 0, bad = k < n && m >= t;
+      if (bad) raise_error(a.err, SAS_ERR_DEVICE_INDEX);
+      const unsigned end_mask = __ballot_sync(0xffffffffu, end);
+      const int first_end = end_mask ? __ffs(end_mask) - 1 : 32;
+      const bool ok = k < n && !bad && m >= 0 && lane < first_end;
+      const unsigned ok_mask = __ballot_sync(0xffffffffu, ok);
+      if (ok) list_s[1 + cnt + __popc(ok_mask & ((1u << lane) - 1u))] = (m << kSlotBits) | (k + 1);
+      cnt += __popc(ok_mask);
+      stop = end_mask != 0;
+    }
+    if (lane == 0) {
+      list_s[0] = t << kSlotBits;
+      nlist_s = 1 + cnt;
+    }
+  } else if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_s), 256);
+    if (lane == 0) {
+      for (int s = 0; s < bdq::kStages; ++s) {
+        mbar_init(smem_u32(&bar_full[s]), 1);
+        mbar_init(smem_u32(&bar_empty[s]), 1);
+      }
+      mbar_init(smem_u32(&bar_fin), 1);
+      fence_barrier_init();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  const int nl = nlist_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmDZ);
+      int issued = 0;
+      for (int i = 0; i < nl; ++i) {
+        const int st = i % bdq::kStages, use = i / bdq::kStages;
+        if (!mbar_wait(smem_u32(&bar_empty[st]), (use & 1) ^ 1, abort_flag, a.err)) break;
+        const uint32_t sk = sbase + st * bdq::kStage, sz = sk + 2 * bdq::kHalfK;
+        const int w = list_s[i];
+        const int krow = int(bh * a.N + size_t(w >> kSlotBits) * kBlock);
+        const long long tile = (slot0 + (w & ((1 << kSlotBits) - 1))) * a.n_hp + hp0;
+        mbar_arrive_expect_tx(smem_u32(&bar_full[st]), uint32_t(2 * bdq::kHalfK + n_tiles * bdq::kTileZ));
+        for (int c = 0; c < 2; ++c) tma_load_2d(sk + c * bdq::kHalfK, &tmK, c * 64, krow, smem_u32(&bar_full[st]));
+        for (int r = 0; r < n_tiles; ++r)
+          tma_load_3d(sz + r * bdq::kTileZ, &tmDZ, 0, 0, int(tile + r), smem_u32(&bar_full[st]));
+        ++issued;
+      }
+      if (*abort_flag) {  // let the copies in flight land before the CTA exits
+        for (int i = max(0, issued - bdq::kStages); i < issued; ++i) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(smem_u32(&bar_full[i % bdq::kStages]), (i / bdq::kStages) & 1) &&
+                 clock64() - t0 < kWaitCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idQ = idesc_bf16_f32(128, 128, 0, 1);  // q rows x d, K = kv tokens; K block MN-major
+      const uint64_t dZ0 = smem_desc_sw128(sbase + 2 * bdq::kHalfK, 16, 1024);
+      const uint64_t dK0 = smem_desc_sw128(sbase, bdq::kHalfK, 1024);
+      bool ok = true;
+      for (int i = 0; ok && i < nl; ++i) {
+        const int st = i % bdq::kStages, use = i / bdq::kStages;
+        if (!(ok = mbar_wait(smem_u32(&bar_full[st]), use & 1, abort_flag, a.err))) break;
+        tc_fence_after();
+        const uint32_t so = st * bdq::kStage;
+        for (int r = 0; r < n_tiles; ++r) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_ss(tmem + r * 128, desc_advance(dZ0, so + r * bdq::kTileZ + k * 32), desc_advance(dK0, so + k * 2048),
+                   idQ, (i > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&bar_empty[st]));
+      }
+      mma_commit(smem_u32(&bar_fin));
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: dQ rows out of TMEM, bf16
+    const int quarter = warp & 3;  // warps 2-5: TMEM lane quarters 2, 3, 0, 1
+    const int row = 32 * quarter + lane;
+    const uint32_t lane_addr = uint32_t(32 * quarter) << 16;
+    bool ok = mbar_wait(smem_u32(&bar_fin), 0, abort_flag, a.err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      for (int r = 0; r < n_tiles; ++r) {
+        const int g = 2 * (hp0 + r) + (row >> 6);
+        const bool valid = g < a.G;  // uniform over the warp: 32 rows of one head
+        const size_t grow = (size_t(b) * a.Hq + size_t(h) * a.G + (valid ? g : 0)) * a.N + size_t(t) * kBlock + (row & 63);
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_addr + r * 128 + ch * 32, v);
+          tmem_wait_ld();
+          if (valid) {
+            uint4* og = reinterpret_cast<uint4*>(a.dq + grow * 128 + ch * 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 o4;
+              o4.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * a.scale, __uint_as_float(v[8 * q4 + 1]) * a.scale);
+              o4.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * a.scale, __uint_as_float(v[8 * q4 + 3]) * a.scale);
+              o4.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * a.scale, __uint_as_float(v[8 * q4 + 5]) * a.scale);
+              o4.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * a.scale, __uint_as_float(v[8 * q4 + 7]) * a.scale);
+              og[q4] = o4;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {
+      const long long t0 = clock64();
+      while (!mbar_try_wait(smem_u32(&bar_fin), 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+long long bwd_dz_tiles(const Shape& sh) {
+  return static_cast<long long>(sh.B) * sh.Hkv * dz_slot_base(sh.NB, sh.K) * ((sh.G + 1) / 2);
+}
+
 cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                    const uint16_t* dO, const float* s, const int32_t* idx, const float* lse_s,
                                    const float* lse_o, const float* drow, const int* rev_off, const int* rev_list,
-                                   const float* rev_lam, float* dl, uint16_t* dq, uint16_t* dk, uint16_t* dv, int* err,
-                                   cudaStream_t st) {
-  CUtensorMap tk, tv, tq3, tdo3, tl, td;
+                                   const float* rev_lam, float* dl, uint16_t* dz, uint16_t* dq, uint16_t* dk,
+                                   uint16_t* dv, int* err, cudaStream_t st) {
+  CUtensorMap tk, tv, tq3, tdo3, tl, td, tdz;
   const uint64_t hq = uint64_t(sh.B) * sh.Hq, rkv = uint64_t(sh.B) * sh.Hkv * sh.N;
   if (!make_tmap_bf16_2d(&tk, k, rkv, 128) || !make_tmap_bf16_2d(&tv, v, rkv, 128) ||
       !make_tmap_bf16_3d_heads(&tq3, q, hq, sh.N) || !make_tmap_bf16_3d_heads(&tdo3, dO, hq, sh.N) ||
       !make_tmap_f32_rows(&tl, lse_o, hq, sh.N) || !make_tmap_f32_rows(&td, drow, hq, sh.N))
+    return cudaErrorInvalidValue;
+  // without a spill region the map is never used; it is encoded over the K cache so that it is valid
+  if (!make_tmap_bf16_tiles(&tdz, dz != nullptr ? static_cast<const void*>(dz) : static_cast<const void*>(k),
+                            dz != nullptr ? uint64_t(bwd_dz_tiles(sh)) : 1))
     return cudaErrorInvalidValue;
   BwdSm100Args a;
   a.rev_off = rev_off;
@@ -826,15 +1040,26 @@ cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const ui
   a.n_hp = (sh.G + 1) / 2;
   a.n_tp = (sh.G + 3) / 4;
   a.scale = sh.scale;
+  a.spill = dz != nullptr ? 1 : 0;
+  a.dz_slots = dz_slot_base(sh.NB, sh.K);
   cudaError_t e;
   auto kv = sh.outside ? bwd_kv_sm100_kernel<true> : bwd_kv_sm100_kernel<false>;
   auto qk = sh.outside ? bwd_q_sm100_kernel<true> : bwd_q_sm100_kernel<false>;
   if ((e = cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, bkv::kSmem)) != cudaSuccess)
     return e;
+  kv<<<dim3(sh.NB, sh.Hkv, sh.B), bkv::kThreads, bkv::kSmem, st>>>(tq3, tk, tv, tdo3, tl, td, tdz, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.spill) {  // dQ from the stored dZ tiles
+    if ((e = cudaFuncSetAttribute(bwd_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bdq::kSmem)) !=
+        cudaSuccess)
+      return e;
+    const int n_pp = (a.n_hp + 1) / 2;
+    bwd_dq_sm100_kernel<<<dim3(sh.NB, sh.Hkv * n_pp, sh.B), bdq::kThreads, bdq::kSmem, st>>>(tk, tdz, a);
+    return cudaGetLastError();
+  }
+  // dQ recomputing S and dP (the small-workspace form)
   if ((e = cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, bq::kSmem)) != cudaSuccess)
     return e;
-  kv<<<dim3(sh.NB, sh.Hkv, sh.B), bkv::kThreads, bkv::kSmem, st>>>(tq3, tk, tv, tdo3, tl, td, a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   qk<<<dim3(sh.NB, sh.Hkv * a.n_hp, sh.B), bq::kThreads, bq::kSmem, st>>>(tk, tv, q, dO, a);
   return cudaGetLastError();
 }

@@ -439,6 +439,19 @@ bool make_tmap_f32_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [tiles, 128, 64] in boxes of one whole tile (128-byte swizzle): the backward's dZ tiles.
+bool make_tmap_bf16_tiles(CUtensorMap* m, const void* base, uint64_t tiles) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {64, 128, tiles};
+  const cuuint64_t strides[2] = {64 * 2, 128 * 64 * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                              const float* s, const int32_t* idx, const float* lse_s, uint16_t* o, float* lse_o,
                              int* err, cudaStream_t st) {

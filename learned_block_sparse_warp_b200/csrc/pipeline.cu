@@ -52,7 +52,7 @@ extern "C" sas_status sas_train_steps_host(const sas_params* p, int n_steps, con
   if (r != SAS_OK) return r;
   if (n_steps < 1 || steps == nullptr || slots == nullptr) return SAS_ERR_INVALID_ARG;
   size_t ws_need = 0;
-  if ((r = sas_bwd_workspace_size(p, &ws_need)) != SAS_OK) return r;
+  if ((r = sas_bwd_workspace_size_min(p, &ws_need)) != SAS_OK) return r;
   for (int k = 0; k < 2 && k < n_steps; ++k) {
     const sas_device_slot& d = slots[k];
     if (!ok16(d.q) || !ok16(d.k) || !ok16(d.v) || !ok16(d.s) || !ok16(d.dO) || !ok16(d.idx) || !ok16(d.lse_s) ||

@@ -16,11 +16,12 @@ cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t*
                              const float* s, const int32_t* idx, const float* lse_s, uint16_t* o, float* lse_o,
                              int* err, cudaStream_t st);
 struct BwdWs;
-size_t bwd_ws_layout(const Shape& sh, void* base, BwdWs* ws);
+size_t bwd_ws_layout(const Shape& sh, bool spill, void* base, BwdWs* ws);
+bool bwd_can_spill(const Shape& sh);
 cudaError_t launch_bwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                            const uint16_t* o, const uint16_t* dO, const float* s, const int32_t* idx,
                            const float* lse_s, const float* lse_o, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* ds,
-                           void* ws, int* err, cudaStream_t st);
+                           void* ws, bool spill, int* err, cudaStream_t st);
 cudaError_t launch_decode(const Shape& sh, const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                           const int32_t* cl, const float* s, const int32_t* idx, const float* lse_s, int n_split,
                           float* o_part, float* lse_part, int* err, cudaStream_t st);
@@ -175,7 +176,16 @@ sas_status sas_bwd_workspace_size(const sas_params* p, size_t* bytes) {
   sas_status r = make_shape(p, &sh);
   if (r != SAS_OK) return r;
   if (bytes == nullptr) return SAS_ERR_INVALID_ARG;
-  *bytes = sas::bwd_ws_layout(sh, nullptr, nullptr);
+  *bytes = sas::bwd_ws_layout(sh, sas::bwd_can_spill(sh), nullptr, nullptr);
+  return SAS_OK;
+}
+
+sas_status sas_bwd_workspace_size_min(const sas_params* p, size_t* bytes) {
+  Shape sh;
+  sas_status r = make_shape(p, &sh);
+  if (r != SAS_OK) return r;
+  if (bytes == nullptr) return SAS_ERR_INVALID_ARG;
+  *bytes = sas::bwd_ws_layout(sh, false, nullptr, nullptr);
   return SAS_OK;
 }
 
@@ -190,10 +200,12 @@ sas_status sas_bwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, co
     return SAS_ERR_INVALID_ARG;
   if (!gate_inputs_ok(sh, s, lse_s) || (sh.gated && !ok_ptr(ds))) return SAS_ERR_INVALID_ARG;
   if (!ok_opt(ds)) return SAS_ERR_INVALID_ARG;
-  const size_t need = sas::bwd_ws_layout(sh, nullptr, nullptr);
+  // the full workspace holds the dZ tiles, which spares the dQ pass recomputing S and dP
+  const bool spill = sas::bwd_can_spill(sh) && ws_bytes >= sas::bwd_ws_layout(sh, true, nullptr, nullptr);
+  const size_t need = sas::bwd_ws_layout(sh, false, nullptr, nullptr);
   if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SAS_ERR_WORKSPACE;
   return from_cuda(sas::launch_bwd_mma(sh, q, k, v, o, dO, sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr,
-                                       lse_o, dq, dk, dv, ds, ws, device_error_word(),
+                                       lse_o, dq, dk, dv, ds, ws, spill, device_error_word(),
                                        static_cast<cudaStream_t>(stream)));
 }
 

@@ -89,6 +89,20 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int x, 
                : "memory");
 }
 
+// 3-D tile store shared -> global (x innermost, all coordinates non-negative), tracked by the
+// issuing thread's bulk-async groups.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, int x, int y, int z, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];\n" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(z), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// Returns once the shared-memory sources of every committed bulk store have been read.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// Returns once every committed bulk store has completed its writes.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
 // 1-D bulk copy global -> shared, completion counted on `bar` (16-byte aligned, size % 16 == 0).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
@@ -219,5 +233,7 @@ bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
 bool make_tmap_bf16_3d_heads(CUtensorMap* m, const void* base, uint64_t heads, uint64_t N);
 // fp32 [rows, N] in boxes of 2 rows x 64 values (host).
 bool make_tmap_f32_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t N);
+// bf16 [tiles, 128, 64]: one box is one whole 16 KB tile of 128 rows x 64 values (128-byte swizzle).
+bool make_tmap_bf16_tiles(CUtensorMap* m, const void* base, uint64_t tiles);
 
 }  // namespace sas

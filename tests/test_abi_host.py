@@ -32,7 +32,8 @@ def _declared():
 
 def test_every_declared_symbol_is_exported():
     names = _declared()
-    assert {"sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd", "sas_bwd_workspace_size", "sas_decode",
+    assert {"sas_topk_select", "sas_gate_lse", "sas_fwd", "sas_bwd", "sas_bwd_workspace_size",
+            "sas_bwd_workspace_size_min", "sas_decode",
             "sas_decode_combine", "sas_get_device_error", "sas_status_string", "sas_version"} <= names
     raw = ctypes.CDLL(sas.LIB_PATH)
     for n in names:
@@ -97,19 +98,30 @@ def test_misaligned_pointers_rejected():
 
 def test_workspace_size_and_check():
     p = _p(batch=2, n_q_heads=8, n_kv_heads=2, seq_len=2048, top_k=8)
+    n_min = sas.sas_bwd_workspace_size_min(p)
     n = sas.sas_bwd_workspace_size(p)
     B, Hq, Hkv, N, d, NB, K = 2, 8, 2, 2048, 128, 32, 8
-    lower = 4 * (B * Hq * N * d + B * Hq * N + B * Hkv * NB * K) + 4 * (B * Hkv * NB * 2 + 2 * B * Hkv * NB * K)
-    assert lower <= n <= lower + 7 * 256
+    # D rows, dl, the reverse index (counts, offsets, entries, gates); no fp32 dQ at d = 128
+    lower = 4 * (B * Hq * N + B * Hkv * NB * K) + 4 * (B * Hkv * NB * 2 + 2 * B * Hkv * NB * K)
+    assert lower <= n_min <= lower + 7 * 256
+    # the full size adds one 16 KB dZ tile per (batch, KV head, query block, attended block, head pair)
+    tiles = B * Hkv * sum(1 + min(K, t) for t in range(NB)) * ((Hq // Hkv + 1) // 2)
+    assert n_min + tiles * 16384 <= n <= n_min + tiles * 16384 + 256
     c = p.c()
     args = [A] * 13
     # too small, unaligned, or missing workspace: SAS_ERR_WORKSPACE before any launch
-    assert lib.sas_bwd(ctypes.byref(c), *args, A, n - 1, None) == WORKSPACE
+    assert lib.sas_bwd(ctypes.byref(c), *args, A, n_min - 1, None) == WORKSPACE
     assert lib.sas_bwd(ctypes.byref(c), *args, A + 16, n, None) == WORKSPACE
     assert lib.sas_bwd(ctypes.byref(c), *args, None, n, None) == WORKSPACE
     size = ctypes.c_size_t(0)
-    assert lib.sas_bwd_workspace_size(None, ctypes.byref(size)) == INVALID
-    assert lib.sas_bwd_workspace_size(ctypes.byref(c), None) == INVALID
+    for fn in (lib.sas_bwd_workspace_size, lib.sas_bwd_workspace_size_min):
+        assert fn(None, ctypes.byref(size)) == INVALID
+        assert fn(ctypes.byref(c), None) == INVALID
+
+
+def test_workspace_d64_has_one_form():
+    p = _p(head_dim=64)
+    assert sas.sas_bwd_workspace_size(p) == sas.sas_bwd_workspace_size_min(p)
 
 
 def test_decode_split_count_checked():
@@ -257,7 +269,8 @@ def test_train_steps_host_checked():
     assert f(ctypes.byref(c), 0, steps, slots, None) == INVALID
     assert f(ctypes.byref(c), 3, None, slots, None) == INVALID
     assert f(ctypes.byref(c), 3, steps, None, None) == INVALID
-    small = (sas.sas_device_slot * 2)(slot, sas.sas_device_slot(*([A] * 14), n - 1))
+    n_min = sas.sas_bwd_workspace_size_min(p)
+    small = (sas.sas_device_slot * 2)(slot, sas.sas_device_slot(*([A] * 14), n_min - 1))
     assert f(ctypes.byref(c), 3, steps, small, None) == WORKSPACE
     bad_slot = (sas.sas_device_slot * 2)(slot, sas.sas_device_slot(*([A] * 13), None, n))
     assert f(ctypes.byref(c), 3, steps, bad_slot, None) == WORKSPACE

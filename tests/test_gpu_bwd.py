@@ -46,10 +46,33 @@ def test_bwd_gate_ablations(case, gate):
     assert max_abs(r["lse_o"], L) < TOL_L
 
 
-def _check_bwd(case, gate):
+D128_CASES = [c for c in CASES if c[4] == 128 and c[5] > 64]
+
+
+@pytest.mark.parametrize("gate", [O.GATE_LOG_SOFTMAX, O.GATE_NONE])
+@pytest.mark.parametrize("case", D128_CASES, ids=[c[0] for c in D128_CASES])
+def test_bwd_small_workspace(case, gate):
+    """With only the smallest workspace the dQ pass recomputes S and dP instead of
+    reading the stored dZ tiles; both forms must match the oracle."""
+    _check_bwd(case, gate, ws_min=True)
+
+
+def test_bwd_workspace_sizes():
+    import learned_block_sparse_warp_b200 as sas
+    # head_dim 128: the full workspace adds one 16 KB dZ tile per (query block, attended block, head pair)
+    p = sas.Params(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, seq_len=1024, top_k=4)
+    slots = sum(1 + min(4, t) for t in range(16))
+    extra = sas.sas_bwd_workspace_size(p) - sas.sas_bwd_workspace_size_min(p)
+    assert 2 * slots * 2 * 16384 <= extra < 2 * slots * 2 * 16384 + 256
+    # head_dim 64 has one form only
+    p64 = sas.Params(batch=1, n_q_heads=2, n_kv_heads=2, head_dim=64, seq_len=1024, top_k=4)
+    assert sas.sas_bwd_workspace_size(p64) == sas.sas_bwd_workspace_size_min(p64)
+
+
+def _check_bwd(case, gate, ws_min=False):
     name, B, Hq, Hkv, d, N, K = case
     w = W.custom(name, batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=N, top_k=K, seed=200 + len(name))
-    x, r, err = run_prefill(w, gate, backward=True)
+    x, r, err = run_prefill(w, gate, backward=True, ws_min=ws_min)
     assert err == 0
     ref_idx, _ = O.prefill_select(x["s"].astype(np.float64), K)
     assert_idx_equal(r["idx"], ref_idx)

@@ -15,8 +15,11 @@ def _sas():
     return sas
 
 
-def run_prefill(w: W.Workload, gate: int, backward: bool = False, idx_override=None):
-    """Runs select + fwd (+ bwd) on the GPU for a small workload; returns host arrays."""
+def run_prefill(w: W.Workload, gate: int, backward: bool = False, idx_override=None, ws_min: bool = False):
+    """Runs select + fwd (+ bwd) on the GPU for a small workload; returns host arrays.
+
+    ws_min: give the backward only its smallest workspace, so that its dQ pass
+    recomputes S and dP instead of reading stored dZ tiles."""
     sas = _sas()
     x = W.prefill_inputs(w, with_do=backward)
     p = sas.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
@@ -24,6 +27,8 @@ def run_prefill(w: W.Workload, gate: int, backward: bool = False, idx_override=N
     q, k, v = bf16_dev(x["q"]), bf16_dev(x["k"]), bf16_dev(x["v"])
     s = f32_dev(x["s"])
     out = sas.empty_prefill_outputs(p, backward=backward)
+    if backward and ws_min:
+        out["ws"] = torch.empty((sas.sas_bwd_workspace_size_min(p),), dtype=torch.uint8, device="cuda")
     sas.sas_topk_select(p, s, out["idx"], out["lse_s"])
     if idx_override is not None:
         out["idx"].copy_(torch.from_numpy(idx_override).cuda())
