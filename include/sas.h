@@ -35,7 +35,13 @@
  *    kernels detect themselves are raised through sas_get_device_error, for
  *    example an index outside the history or a bounded wait that expired.
  *  - Calls keep no state between them and may be issued from several host
- *    threads, on different streams.
+ *    threads, on different streams, with two exceptions. Each device has one
+ *    error word, shared by every caller: sas_get_device_error reads and
+ *    clears it, so one caller's read also clears what another caller's
+ *    kernels raised. And sas_decode_noalloc shares one fixed scratch array
+ *    per device (see there). The library looks up the device addresses of
+ *    both once per device and keeps them: after cudaDeviceReset on a device,
+ *    unload and reload the library before calling it on that device.
  *
  * Shapes (sas_params): B = batch, Hq = n_q_heads, Hkv = n_kv_heads,
  * G = Hq / Hkv (GQA group), d = head_dim, N = seq_len, b = block (64),
@@ -334,7 +340,8 @@ SAS_API sas_status sas_decode_select_scored(const sas_params* p, const sas_bf16*
  *    library holds these 16 MiB until the process exits.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current). Make that first call
- *    before any stream capture on that device.
+ *    before any stream capture on that device. The address is kept for the
+ *    life of the library: after cudaDeviceReset, reload the library.
  *  - Every call shares the one array per device. Calls that overlap on the
  *    GPU (other streams, other host threads) race on it; the caller must
  *    order them. Each call writes all the scratch it reads, so nothing needs
@@ -412,7 +419,9 @@ SAS_API sas_status sas_selftest_wait_timeout(void* stream);
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device. *code is SAS_OK when no kernel raised an error since the
  * last read, else the first sas_status a kernel raised (SAS_ERR_TIMEOUT or
- * SAS_ERR_DEVICE_INDEX). */
+ * SAS_ERR_DEVICE_INDEX). The word is one per device and shared by every
+ * caller of the library in the process: a kernel of any caller may have
+ * raised it, and this read clears it for all of them. */
 SAS_API sas_status sas_get_device_error(void* stream, int* code);
 
 /* Static, human-readable name of a status code. */
