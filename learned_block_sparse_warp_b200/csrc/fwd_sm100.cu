@@ -8,22 +8,26 @@
 //
 // One CTA owns one (batch, KV head, query block) and up to four query heads
 // of the group. That is 256 rows, packed as two M = 128 tiles of two heads
-// each, so every gathered K/V block serves four heads (GQA packing). Roles:
+// each, so every gathered K/V block serves four heads (GQA packing). A step
+// is one gathered 64-token block. Roles:
 //   warp 0       builds the block list [t, I_t...], then issues TMA loads:
-//                the Q rows once, then the selected K/V blocks two at a time
-//                (N = 128) into a 2-stage shared-memory ring. Blocks are
-//                gathered by index with no copy in HBM.
-//   warp 1       allocates 512 TMEM columns and issues every tcgen05.mma:
-//                S_r = Q_r Kᵀ (SS, fp32 in TMEM), then O_r += P_r V (TS:
-//                P_r read from TMEM).
+//                the Q rows once, then each selected K/V block into a
+//                4-stage shared-memory ring. Blocks are gathered by index
+//                with no copy in HBM.
+//   warps 1, 3   one MMA-issuing thread per tile (warp 1 also allocates the
+//                512 TMEM columns): S_r(b) = Q_r K_bᵀ (SS, fp32 in TMEM), then
+//                O_r += P_r(b) V_b (TS: P read from TMEM).
 //   warps 4-7    softmax of tile 0; warps 8-11 softmax of tile 1. Each thread
-//                owns one row: it reads S from TMEM, adds the block's
-//                log-gate (one scalar per 64 columns), masks the current
-//                block causally, updates the row max and sum, and writes
-//                bf16 P back over the consumed S columns. O is rescaled in
-//                TMEM only when the row max grows by more than 2^8, so the
-//                result is exact and rescales are rare.
-// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+//                owns one row: it reads the block's 64 logits from TMEM,
+//                masks the current block causally, adds the block's log-gate,
+//                updates the row max and sum, and writes bf16 P back over the
+//                consumed S columns. O is rescaled in TMEM only when the row
+//                max grows by more than 2^8, so the result is exact and
+//                rescales are rare.
+// Each tile has two 64-column S buffers: S of block b + 1 is computed while
+// the softmax works on block b and PV of block b − 1 runs, so no tile waits
+// for its own PV before its next S.
+// TMEM, tile r at column 256 r: S buffers [0, 64) and [64, 128), O [128, 256).
 // Every mbarrier wait is bounded and raises SAS_ERR_TIMEOUT instead of hanging.
 #include <mutex>
 
@@ -32,13 +36,14 @@
 namespace sas {
 
 namespace fsm {
-constexpr int kThreads = 384;                    // 0 TMA, 1 and 3 MMA (one per tile), 4-11 softmax
-constexpr int kStages = 2;
-constexpr int kHalf = 128 * 128;                 // one d-half of a 128-row tile: 128 rows x 128 B
-constexpr int kQBytes = 4 * kHalf;               // 2 tiles x 2 d-halves
-constexpr int kStageBytes = 4 * kHalf;           // K and V, 2 d-halves each, 128 token rows
+constexpr int kThreads = 384;            // 0 TMA, 1 and 3 MMA (one per tile), 4-11 softmax
+constexpr int kStages = 4;               // one gathered K/V block per stage
+constexpr int kHalf = 128 * 128;         // one d-half of a 128-row Q tile: 128 rows x 128 B
+constexpr int kQBytes = 4 * kHalf;       // 2 tiles x 2 d-halves
+constexpr int kHalfKV = 64 * 128;        // one d-half of a 64-row K or V block
+constexpr int kStageBytes = 4 * kHalfKV;  // K and V of one block, two d-halves each
 constexpr int kSmemBytes = kQBytes + kStages * kStageBytes + 1024;  // + room to align to 1 KB
-constexpr float kRescale = 8.0f;                 // log2 headroom before O is rescaled
+constexpr float kRescale = 8.0f;         // log2 headroom before O is rescaled
 }  // namespace fsm
 
 struct FwdSm100Args {
@@ -54,6 +59,16 @@ struct FwdSm100Args {
 
 // kOut: the gate weights the values after a softmax over the plain logits
 // (SAS_GATE_SOFTMAX_OUTSIDE) instead of entering the logits as log g.
+//
+// Barriers, for tile r and block b (c = b & 1 selects the S buffer):
+//   producer   waits empty[st] (block b − 4), loads K_b, V_b        -> full[st]
+//   MMA r      waits full of b + 1 and pv[c'] (PV of b − 1, the buffer S(b + 1)
+//              reuses), issues S(b + 1)                               -> s[c']
+//              waits p[c] (P of b in TMEM), issues PV(b)             -> pv[c], empty[st]
+//   softmax r  waits s[c], writes P(b)                                -> p[c]
+//              (waits pv of b − 1 before a rare rescale of O)
+// No waiter can fall two phases behind: every barrier's next phase needs the
+// waiter's own next action first.
 template <bool kOut>
 __global__ void __launch_bounds__(fsm::kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -63,13 +78,8 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
   __shared__ int list_s[kMaxTopK + 1];
   __shared__ float lam_s[kMaxTopK + 1];
   __shared__ int nlist_s;
-  // bar_turn[r]: tile r's softmax may run its exponentials. The two tiles take
-  // turns, so one tile's exponentials overlap the other tile's MMAs instead of
-  // both contending for the SM's exponential units at once.
-  // bar_p[r] / bar_pb[r]: tile r's P of the pair's first / second 64-column block is in TMEM,
-  // so the PV of the first block starts while the second block's exponentials run.
-  __shared__ __align__(8) uint64_t bar_q, bar_full[fsm::kStages], bar_empty[fsm::kStages], bar_s[2], bar_p[2],
-      bar_pb[2], bar_o[2], bar_fin, bar_turn[2];
+  __shared__ __align__(8) uint64_t bar_q, bar_full[fsm::kStages], bar_empty[fsm::kStages], bar_s[2][2], bar_p[2][2],
+      bar_pv[2][2], bar_fin;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
 
@@ -99,15 +109,13 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         mbar_init(smem_u32(&bar_full[s]), 1);
         mbar_init(smem_u32(&bar_empty[s]), n_tiles);  // one commit per tile's MMA thread
       }
-      for (int r = 0; r < 2; ++r) {
-        mbar_init(smem_u32(&bar_s[r]), 1);
-        mbar_init(smem_u32(&bar_p[r]), 128);
-        mbar_init(smem_u32(&bar_pb[r]), 128);
-        mbar_init(smem_u32(&bar_o[r]), 1);
-      }
+      for (int r = 0; r < 2; ++r)
+        for (int c = 0; c < 2; ++c) {
+          mbar_init(smem_u32(&bar_s[r][c]), 1);
+          mbar_init(smem_u32(&bar_p[r][c]), 128);
+          mbar_init(smem_u32(&bar_pv[r][c]), 1);
+        }
       mbar_init(smem_u32(&bar_fin), n_tiles);
-      mbar_init(smem_u32(&bar_turn[0]), 4);  // one arrival per softmax warp of the other tile
-      mbar_init(smem_u32(&bar_turn[1]), 4);
       fence_barrier_init();
     }
   }
@@ -116,7 +124,6 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_s;
   const int nl = nlist_s;
-  const int n_pairs = (nl + 1) / 2;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -132,25 +139,22 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
           tma_load_2d(sQ + (r * 2 + c) * fsm::kHalf + half * 8192, &tmQ, c * 64, row, smem_u32(&bar_q));
       }
       int issued = 0;
-      for (int p = 0; p < n_pairs; ++p) {
-        const int st = p % fsm::kStages, use = p / fsm::kStages;
+      for (int i = 0; i < nl; ++i) {
+        const int st = i % fsm::kStages, use = i / fsm::kStages;
         if (!mbar_wait(smem_u32(&bar_empty[st]), (use & 1) ^ 1, abort_flag, a.err)) break;
-        const int nb = min(2, nl - 2 * p);
-        mbar_arrive_expect_tx(smem_u32(&bar_full[st]), uint32_t(nb) * 4u * 8192u);
-        const uint32_t sk = sKV + st * fsm::kStageBytes, sv = sk + 2 * fsm::kHalf;
-        for (int bb = 0; bb < nb; ++bb) {
-          const int row = int(bh * a.N + size_t(list_s[2 * p + bb]) * kBlock);
-          for (int c = 0; c < 2; ++c) {
-            tma_load_2d(sk + c * fsm::kHalf + bb * 8192, &tmK, c * 64, row, smem_u32(&bar_full[st]));
-            tma_load_2d(sv + c * fsm::kHalf + bb * 8192, &tmV, c * 64, row, smem_u32(&bar_full[st]));
-          }
+        mbar_arrive_expect_tx(smem_u32(&bar_full[st]), 4u * 8192u);
+        const uint32_t sk = sKV + st * fsm::kStageBytes, sv = sk + 2 * fsm::kHalfKV;
+        const int row = int(bh * a.N + size_t(list_s[i]) * kBlock);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_2d(sk + c * fsm::kHalfKV, &tmK, c * 64, row, smem_u32(&bar_full[st]));
+          tma_load_2d(sv + c * fsm::kHalfKV, &tmV, c * 64, row, smem_u32(&bar_full[st]));
         }
         ++issued;
       }
       if (*abort_flag) {  // let the loads already in flight land before the CTA exits
-        for (int p = max(0, issued - fsm::kStages); p < issued; ++p) {
+        for (int i = max(0, issued - fsm::kStages); i < issued; ++i) {
           const long long t0 = clock64();
-          while (!mbar_try_wait(smem_u32(&bar_full[p % fsm::kStages]), (p / fsm::kStages) & 1) &&
+          while (!mbar_try_wait(smem_u32(&bar_full[i % fsm::kStages]), (i / fsm::kStages) & 1) &&
                  clock64() - t0 < kWaitCycles) {
           }
         }
@@ -158,45 +162,46 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
     }
   } else if ((warp == 1 || warp == 3) && (warp >> 1) < n_tiles) {
     // ------------------------------------------------------------ MMA issuers, one thread per tile
-    // (each tile's chain S → softmax → PV is latency-bound; two threads let the
-    // two tiles' MMAs overlap)
     if (lane == 0) {
       const int r = warp >> 1;
-      const uint32_t idS2 = idesc_bf16_f32(128, 128, 0, 0), idS1 = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
+      const uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);   // q rows x kv, K = d
+      const uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);  // q rows x d, K = kv; V MN-major
+      // descriptors are built once; a stage or K step only moves the start address
       const uint64_t dQ0 = smem_desc_sw128(sQ + r * 2 * fsm::kHalf, 16, 1024);
       const uint64_t dK0 = smem_desc_sw128(sKV, 16, 1024);
-      const uint64_t dV0 = smem_desc_sw128(sKV + 2 * fsm::kHalf, fsm::kHalf, 1024);
-      const uint32_t tS = tmem + r * 128, tO = tmem + 256 + r * 128;
-      bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, a.err);
-      tc_fence_after();
-      for (int p = 0; ok && p < n_pairs; ++p) {
-        const int st = p % fsm::kStages, use = p / fsm::kStages;
-        if (!(ok = mbar_wait(smem_u32(&bar_full[st]), use & 1, abort_flag, a.err))) break;
-        if (p > 0) {  // PV(p-1) reads P from the columns that S(p) overwrites
-          if (!(ok = mbar_wait(smem_u32(&bar_o[r]), (p - 1) & 1, abort_flag, a.err))) break;
-        }
-        tc_fence_after();
-        const int nb = min(2, nl - 2 * p);
-        const uint32_t so = st * fsm::kStageBytes;
+      const uint64_t dV0 = smem_desc_sw128(sKV + 2 * fsm::kHalfKV, fsm::kHalfKV, 1024);
+      const uint32_t tT = tmem + r * 256, tO = tT + 128;
+      auto issue_s = [&](const int i) {  // S of block i into buffer i & 1
+        const uint32_t so = (i % fsm::kStages) * fsm::kStageBytes;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t oc = (k >> 2) * fsm::kHalf + (k & 3) * 32;
-          mma_ss(tS, desc_advance(dQ0, oc), desc_advance(dK0, so + oc), nb == 2 ? idS2 : idS1, k > 0 ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&bar_s[r]));
-        if (!(ok = mbar_wait(smem_u32(&bar_p[r]), p & 1, abort_flag, a.err))) break;
-        tc_fence_after();
-        for (int jj = 0; jj < 4; ++jj)  // the first block's 64 tokens
-          mma_ts(tO, tS + jj * 8, desc_advance(dV0, so + jj * 2048), idPV, (p > 0 || jj > 0) ? 1u : 0u);
-        if (nb > 1) {  // the second block's, once its P is in (every pair but an odd last one)
-          if (!(ok = mbar_wait(smem_u32(&bar_pb[r]), p & 1, abort_flag, a.err))) break;
+        for (int k = 0; k < 8; ++k)
+          mma_ss(tT + (i & 1) * 64, desc_advance(dQ0, (k >> 2) * fsm::kHalf + (k & 3) * 32),
+                 desc_advance(dK0, so + (k >> 2) * fsm::kHalfKV + (k & 3) * 32), idS, k > 0 ? 1u : 0u);
+        mma_commit(smem_u32(&bar_s[r][i & 1]));
+      };
+      bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, a.err);
+      ok = ok && mbar_wait(smem_u32(&bar_full[0]), 0, abort_flag, a.err);
+      tc_fence_after();
+      if (ok) issue_s(0);
+      for (int i = 0; ok && i < nl; ++i) {
+        if (i + 1 < nl) {
+          const int n = i + 1;
+          if (!(ok = mbar_wait(smem_u32(&bar_full[n % fsm::kStages]), (n / fsm::kStages) & 1, abort_flag, a.err)))
+            break;
+          // PV of block n − 2 read its P from the buffer that S(n) overwrites
+          if (n >= 2 && !(ok = mbar_wait(smem_u32(&bar_pv[r][n & 1]), ((n - 2) >> 1) & 1, abort_flag, a.err)))
+            break;
           tc_fence_after();
-          for (int jj = 4; jj < 8; ++jj)
-            mma_ts(tO, tS + jj * 8, desc_advance(dV0, so + jj * 2048), idPV, 1u);
+          issue_s(n);
         }
-        mma_commit(smem_u32(&bar_o[r]));
-        mma_commit(smem_u32(&bar_empty[st]));
+        if (!(ok = mbar_wait(smem_u32(&bar_p[r][i & 1]), (i >> 1) & 1, abort_flag, a.err))) break;
+        tc_fence_after();
+        const uint32_t sv = (i % fsm::kStages) * fsm::kStageBytes;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)  // P(i) packed over the first 32 columns of its S buffer
+          mma_ts(tO, tT + (i & 1) * 64 + jj * 8, desc_advance(dV0, sv + jj * 2048), idPV, (i > 0 || jj > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&bar_pv[r][i & 1]));
+        mma_commit(smem_u32(&bar_empty[i % fsm::kStages]));
       }
       mma_commit(smem_u32(&bar_fin));
     }
@@ -206,58 +211,38 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
     const int quarter = warp & 3;
     const int row = 32 * quarter + lane;
     const uint32_t lane_addr = uint32_t(32 * quarter) << 16;
-    const uint32_t tS = tmem + lane_addr + r * 128, tO = tmem + lane_addr + 256 + r * 128;
+    const uint32_t tT = tmem + lane_addr + r * 256, tO = tT + 128;
     const int qpos = row & 63;
     const float sc2 = a.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int p = 0; p < n_pairs; ++p) {
-      ok = mbar_wait(smem_u32(&bar_s[r]), p & 1, abort_flag, a.err);
+    for (int i = 0; i < nl; ++i) {
+      const uint32_t tS = tT + (i & 1) * 64;
+      ok = mbar_wait(smem_u32(&bar_s[r][i & 1]), (i >> 1) & 1, abort_flag, a.err);
       if (!__all_sync(0xffffffffu, ok)) {  // TMEM loads below are warp-collective
         ok = false;
         break;
       }
       tc_fence_after();
-      const int nb = min(2, nl - 2 * p);
-      // log2 g of the pair's two blocks, as a logit bias (the gate outside the softmax adds none)
-      const float lamA = kOut ? 0.f : lam_s[2 * p], lamB = (kOut || nb < 2) ? 0.f : lam_s[2 * p + 1];
-      const bool diag = (p == 0);  // block A of pair 0 is the causal current block
-      // The pair's S row (up to 128 columns) comes out of TMEM in four loads and
-      // one wait, and stays in registers. Raw row max per 64-column block; the
-      // scale and gate are applied to the max. The current block is causal.
-      uint32_t v[128];
+      // log2 g of the block as a logit bias (the gate outside the softmax adds none)
+      const float lam = kOut ? 0.f : lam_s[i];
+      uint32_t v[64];
       tmem_ld32(tS, v);
       tmem_ld32(tS + 32, v + 32);
-      if (nb > 1) {
-        tmem_ld32(tS + 64, v + 64);
-        tmem_ld32(tS + 96, v + 96);
-      }
       tmem_wait_ld();
-      if (diag) {
+      if (i == 0) {  // the current block is causal
 #pragma unroll
         for (int e = 0; e < 64; ++e) v[e] = e <= qpos ? v[e] : __float_as_uint(-INFINITY);
       }
-      float rmA = -INFINITY, rmB = -INFINITY;
-      {
-        float m0 = -INFINITY, m1 = -INFINITY;
+      float mm[8];
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          m0 = fmaxf(m0, __uint_as_float(v[e]));
-          m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
-        }
-        rmA = fmaxf(m0, m1);
-      }
-      if (nb > 1) {
-        float m0 = -INFINITY, m1 = -INFINITY;
+      for (int c = 0; c < 8; ++c) mm[c] = fmaxf(__uint_as_float(v[c]), __uint_as_float(v[c + 8]));
 #pragma unroll
-        for (int e = 64; e < 128; e += 2) {
-          m0 = fmaxf(m0, __uint_as_float(v[e]));
-          m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
-        }
-        rmB = fmaxf(m0, m1);
-      }
-      float mx = rmA == -INFINITY ? -INFINITY : fmaf(rmA, sc2, lamA);
-      if (nb > 1) mx = fmaxf(mx, fmaf(rmB, sc2, lamB));
+      for (int e = 16; e < 64; e += 8)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mm[c] = fmaxf(mm[c], __uint_as_float(v[e + c]));
+      const float rm = fmaxf(fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])), fmaxf(fmaxf(mm[4], mm[5]), fmaxf(mm[6], mm[7])));
+      const float mx = rm == -INFINITY ? -INFINITY : fmaf(rm, sc2, lam);
       // The stabiliser moves only when the row max grows by more than 2^8. The
       // decision is per row, but the TMEM round trip that rescales O is a
       // warp-collective instruction, so a warp runs it whenever any of its rows
@@ -269,29 +254,18 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         l *= alpha;
         m_used = mx;
       }
-      // Turn order: tile 0 pair 0, tile 1 pair 0, tile 0 pair 1, ... Tile 0 waits for
-      // tile 1's turn of pair p - 1, tile 1 for tile 0's turn of pair p. Neither
-      // barrier can run a phase ahead: its next phase needs the waiter's own turn.
-      if (n_tiles == 2 && (r == 1 || p > 0)) {
-        const bool got = mbar_wait(smem_u32(&bar_turn[r]), (r == 0 ? p - 1 : p) & 1, abort_flag, a.err);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-      }
-      // probabilities, row sum, bf16 P over the S columns (all read above), one 64-column
-      // block at a time: block ch2's P goes to TMEM columns [32 ch2, 32 ch2 + 32)
-      auto block_p = [&](const int ch2) {
-        const float off = (ch2 == 0 ? lamA : lamB) - m_used;  // p = 2^(S·sc2 + λ − m)
+      // probabilities, row sum, bf16 P over the S columns just read
+      {
+        const float off = lam - m_used;  // p = 2^(S·sc2 + λ − m)
         uint32_t pk[32];
         float s0 = 0.f, s1 = 0.f;
         // gate outside: the row sum takes p, the values take g·p
         __nv_bfloat162 gw2;
-        if constexpr (kOut) gw2 = __float2bfloat162_rn(fast_exp2(lam_s[2 * p + ch2]));
+        if constexpr (kOut) gw2 = __float2bfloat162_rn(fast_exp2(lam_s[i]));
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(v[64 * ch2 + 2 * e]), sc2, off));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(v[64 * ch2 + 2 * e + 1]), sc2, off));
+          const float p0 = fast_exp2(fmaf(__uint_as_float(v[2 * e]), sc2, off));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), sc2, off));
           s0 += p0;
           s1 += p1;
           pk[e] = pack_bf16x2(p0, p1);
@@ -301,20 +275,16 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
           }
         }
         l += s0 + s1;
-        tmem_st32(tS + ch2 * 32, pk);
-      };
-      // the turn guards the exponentials only: it passes as soon as the last block's are done
-      auto pass_turn = [&]() {
-        if (n_tiles == 2) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&bar_turn[r ^ 1]));
+        tmem_st32(tS, pk);
+      }
+      if (i > 0 && __any_sync(0xffffffffu, grow)) {
+        // O holds PV of the earlier blocks once PV(i − 1) has completed
+        ok = mbar_wait(smem_u32(&bar_pv[r][(i - 1) & 1]), ((i - 1) >> 1) & 1, abort_flag, a.err);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
         }
-      };
-      block_p(0);
-      if (nb == 1) pass_turn();
-      if (p > 0 && __any_sync(0xffffffffu, grow)) {
-        // O holds PV of earlier pairs, complete because S_r(p) completed after it. It is
-        // rescaled before the first block's PV of this pair is released, 16 columns at a time.
+        tc_fence_after();
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t w[16];
           tmem_ld16(tO + ch * 16, w);
@@ -326,16 +296,9 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bar_p[r]));
-      if (nb > 1) {
-        block_p(1);
-        pass_turn();
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(smem_u32(&bar_pb[r]));
-      }
+      mbar_arrive(smem_u32(&bar_p[r][i & 1]));
     }
-    if (ok) ok = mbar_wait(smem_u32(&bar_o[r]), (n_pairs - 1) & 1, abort_flag, a.err);
+    if (ok) ok = mbar_wait(smem_u32(&bar_pv[r][(nl - 1) & 1]), ((nl - 1) >> 1) & 1, abort_flag, a.err);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
@@ -346,17 +309,17 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         const float inv = 1.f / l;
         uint4* og = reinterpret_cast<uint4*>(a.o + orow * 128);
         for (int ch = 0; ch < 4; ++ch) {
-          uint32_t v[32];
-          tmem_ld32(tO + ch * 32, v);
+          uint32_t w[32];
+          tmem_ld32(tO + ch * 32, w);
           tmem_wait_ld();
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
-            og[ch * 4 + q4] = w;
+            uint4 x;
+            x.x = pack_bf16x2(__uint_as_float(w[8 * q4 + 0]) * inv, __uint_as_float(w[8 * q4 + 1]) * inv);
+            x.y = pack_bf16x2(__uint_as_float(w[8 * q4 + 2]) * inv, __uint_as_float(w[8 * q4 + 3]) * inv);
+            x.z = pack_bf16x2(__uint_as_float(w[8 * q4 + 4]) * inv, __uint_as_float(w[8 * q4 + 5]) * inv);
+            x.w = pack_bf16x2(__uint_as_float(w[8 * q4 + 6]) * inv, __uint_as_float(w[8 * q4 + 7]) * inv);
+            og[ch * 4 + q4] = x;
           }
         }
         if (a.lse_o != nullptr) a.lse_o[orow] = (m_used + log2f(l)) * kLn2;
