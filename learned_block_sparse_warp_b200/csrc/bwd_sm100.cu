@@ -12,7 +12,7 @@
 //   bwd_kv_sm100_kernel  one CTA per (batch, KV head, KV block j). It walks the
 //       query blocks that attend j (its own diagonal block first, then the
 //       reverse index), two query heads (128 rows) per step. S = Q Kᵀ and
-//       dP = dO Vᵀ land in double-buffered TMEM. The softmax-gradient warps
+//       dP = dO Vᵀ land in a three-deep TMEM ring. The softmax-gradient warps
 //       write P and dZ as bf16 rows, 128-byte swizzled, into shared memory.
 //       dVᵀ += dOᵀ P and dKᵀ += Qᵀ dZ then accumulate in TMEM as M = 128
 //       (d-major) MMAs with MN-major operands, so dK_j and dV_j stay on chip
@@ -82,7 +82,7 @@ struct Meta {
   float lam2;
 };
 struct Ctl {
-  uint64_t bar_kv, fq[kNQ], eq[kNQ], fo[kNO], eo[kNO], bs[2], bd[2], bp[2], bz[2], pf, zf, fin;
+  uint64_t bar_kv, fq[kNQ], eq[kNQ], fo[kNO], eo[kNO], bs[3], bd[3], bp[3], bz[3], pf, zf, fin;
   Meta meta[kNQ];
   float red_s[2][kSoftWarps];
   uint32_t tmem;
@@ -142,20 +142,21 @@ struct EntryRing {
 // softmax-gradient warps (four per SM sub-partition) write P as soon as S
 // allows, so dVᵀ starts before dP is consumed, then dZ.
 //
-// Per step i, with q = i % 3, o = i % 2 and b = i & 1 (the TMEM S/dP buffer):
+// Per step i, with q = i % 3, o = i % 2 and b = i % 3 (the TMEM S/dP buffer):
 //   Q producer   waits eq[q] (step i - 3), loads Q, L        -> fq[q]
 //   dO producer  waits eo[o] (step i - 2), loads dO, D       -> fo[o]
-//   S            waits fq[q], bp[b] (step i - 2)             -> bs[b], eq[q]
-//   dP           waits fo[o], bz[b] (step i - 2)             -> bd[b], eo[o]
+//   S            waits fq[q], bp[b] (step i - 3)             -> bs[b], eq[q]
+//   dP           waits fo[o], bz[b] (step i - 3)             -> bd[b], eo[o]
 //   softmax      waits fq[q], fo[o], bs[b], reads L, D and the entry;
 //                waits pf (step i - 1), writes P  -> bp[b]
 //                waits bd[b] and zf (step i - 1), writes dZ -> bz[b]
 //   dVᵀ          waits fo[o], bp[b]                          -> pf, eo[o]
 //   dKᵀ          waits fq[q], bz[b]                          -> zf, eq[q]
 //                and, when spilling, stores the dZ tile     -> zf (second arrival, once it is read)
-// bp and bz are per TMEM buffer because the S and dP issuers wait two steps
-// back; with one barrier they could fall two phases behind. Every other
-// waiter's next phase needs the waiter's own next action first.
+// bp and bz are per TMEM buffer because the S and dP issuers wait three steps
+// back; with one barrier they could fall phases behind. Every other waiter's
+// next phase needs the waiter's own next action first. The three-deep ring
+// lets S and dP run up to three steps ahead of the softmax-gradient warps.
 // kOut: the gate weights the values after a softmax over the plain logits
 // (SAS_GATE_SOFTMAX_OUTSIDE): dVᵀ takes g·P, dZ = P·(g·dP − D) and
 // dl = Σ P·g·dP (= g ∂/∂g) instead of Σ dZ.
@@ -207,7 +208,7 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
         mbar_init(smem_u32(&C.fo[s]), 1);
         mbar_init(smem_u32(&C.eo[s]), 2);
       }
-      for (int r = 0; r < 2; ++r) {
+      for (int r = 0; r < 3; ++r) {
         mbar_init(smem_u32(&C.bs[r]), 1);
         mbar_init(smem_u32(&C.bd[r]), 1);
         mbar_init(smem_u32(&C.bp[r]), bkv::kSoftWarps);
@@ -223,8 +224,8 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = C.tmem;
-  // TMEM columns: S buffers 0 / 64, dP buffers 128 / 192, dVᵀ 256, dKᵀ 320
-  constexpr uint32_t kColDV = 256, kColDK = 320;
+  // TMEM columns: S buffers 0 / 64 / 128, dP buffers 192 / 256 / 320, dVᵀ 384, dKᵀ 448
+  constexpr uint32_t kColDV = 384, kColDK = 448;
 
   if (warp == 0 || warp == bkv::kWarpProdO) {
     // ------------------------------------------------------------ TMA producers
@@ -303,14 +304,14 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
       // Descriptors are built once; a slot or K step only moves the start address.
       const uint64_t dA = smem_desc_sw128(is_s ? sQ : sO, 16, 1024);
       const uint64_t dB = smem_desc_sw128(is_s ? sK : sV, 16, 1024);
-      const uint32_t tD = tmem + (is_s ? 0u : 128u);
+      const uint32_t tD = tmem + (is_s ? 0u : 192u);
       bool ok = mbar_wait(smem_u32(&C.bar_kv), 0, abort_flag, a.err);
       tc_fence_after();
       for (int i = 0; ok && i < n_steps; ++i) {
-        const int st = i % nslot, use = i / nslot, sb = i & 1;
+        const int st = i % nslot, use = i / nslot, sb = i % 3;
         if (!(ok = mbar_wait(smem_u32(is_s ? &C.fq[st] : &C.fo[st]), use & 1, abort_flag, a.err))) break;
-        // the softmax-gradient warps have read S / dP of step i - 2 from this buffer
-        if (i >= 2 && !(ok = mbar_wait(smem_u32(is_s ? &C.bp[sb] : &C.bz[sb]), ((i - 2) >> 1) & 1, abort_flag, a.err)))
+        // the softmax-gradient warps have read S / dP of step i - 3 from this buffer
+        if (i >= 3 && !(ok = mbar_wait(smem_u32(is_s ? &C.bp[sb] : &C.bz[sb]), ((i - 3) / 3) & 1, abort_flag, a.err)))
           break;
         tc_fence_after();
         const uint32_t so = st * bkv::kTile;
@@ -334,9 +335,9 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
       const uint32_t tG = tmem + (is_v ? kColDV : kColDK);
       bool ok = true;
       for (int i = 0; ok && i < n_steps; ++i) {
-        const int st = i % nslot, use = i / nslot, sb = i & 1;
+        const int st = i % nslot, use = i / nslot, sb = i % 3;
         if (!(ok = mbar_wait(smem_u32(is_v ? &C.fo[st] : &C.fq[st]), use & 1, abort_flag, a.err))) break;
-        if (!(ok = mbar_wait(smem_u32(is_v ? &C.bp[sb] : &C.bz[sb]), (i >> 1) & 1, abort_flag, a.err))) break;
+        if (!(ok = mbar_wait(smem_u32(is_v ? &C.bp[sb] : &C.bz[sb]), (i / 3) & 1, abort_flag, a.err))) break;
         tc_fence_after();
         // read before the MMAs: their commit on eq lets the producer refill this Q slot and its meta
         const bkv::Meta m = is_v ? bkv::Meta{0, 0, 0, 0.f} : C.meta[st];
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
     // After an abort a warp keeps walking the steps without touching TMEM or
     // shared tiles, so that every softmax warp still meets named barrier 1.
     for (int i = 0; i < n_steps; ++i) {
-      const int qs = i % bkv::kNQ, os = i % bkv::kNO, sb = i & 1;
+      const int qs = i % bkv::kNQ, os = i % bkv::kNO, sb = i % 3;
       const int e = i / a.n_hp, hp = i % a.n_hp;
       const bool diag = (e == 0);
       // Everything this step reads from the Q and dO slots (L, D, the entry) is
@@ -384,7 +385,7 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
       if (ok) {
         ok = mbar_wait(smem_u32(&C.fq[qs]), (i / bkv::kNQ) & 1, abort_flag, a.err);
         ok = ok && mbar_wait(smem_u32(&C.fo[os]), (i / bkv::kNO) & 1, abort_flag, a.err);
-        ok = ok && mbar_wait(smem_u32(&C.bs[sb]), (i >> 1) & 1, abort_flag, a.err);
+        ok = ok && mbar_wait(smem_u32(&C.bs[sb]), (i / 3) & 1, abort_flag, a.err);
         ok = __all_sync(0xffffffffu, ok);
       }
       const bkv::Meta m = C.meta[qs];
@@ -426,13 +427,13 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&C.bp[sb]));
-        ok = mbar_wait(smem_u32(&C.bd[sb]), (i >> 1) & 1, abort_flag, a.err);
+        ok = mbar_wait(smem_u32(&C.bd[sb]), (i / 3) & 1, abort_flag, a.err);
         ok = __all_sync(0xffffffffu, ok);
       }
       if (ok) {
         tc_fence_after();
         uint32_t vp[16];
-        tmem_ld16(tmem + lane_addr + 128 + sb * 64 + cg * 16, vp);
+        tmem_ld16(tmem + lane_addr + 192 + sb * 64 + cg * 16, vp);
         tmem_wait_ld();
         float zr[16];
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
