@@ -419,7 +419,7 @@ def run_gpu(args, rank, world, local_rank):
         del x, out
         torch.cuda.empty_cache()
 
-    # ---------------- decode: select, split-K, merge; L2 flushed before every timed step ----------------
+    # ---------------- decode: select, split-K, merge, over rotating selections ----------------
     if args.only in ("all", "decode") and not args.no_decode:
         wd = W.WORKLOADS[DECODE]
         pd = sas.Params(batch=wd.batch, n_q_heads=wd.n_q_heads, n_kv_heads=wd.n_kv_heads, head_dim=wd.head_dim,
@@ -432,25 +432,41 @@ def run_gpu(args, rank, world, local_rank):
         flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
         flush_sink = torch.empty((), dtype=torch.float32, device=dev)
 
-        def dstep_eager():
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-            ev[0].record(stream)
-            sas.decode_step(pd, xd["q"], xd["k"], xd["v"], xd["cache_len"], xd["s"], n_split, od, stream=stream)
-            ev[1].record(stream)
-            return ev
-
-        # a serving loop replays the captured step. The per-kernel breakdown launches each kernel on
-        # its own between two events, with the L2 flush queued before it: the launch overlaps the flush,
-        # so the event pair spans the kernel and not a graph launch
-        step_graph = sas.DecodeGraph(pd, xd["q"], xd["k"], xd["v"], xd["cache_len"], xd["s"], n_split, od,
-                                     stream=stream)
+        # Timing. A serving loop replays the captured step. Each figure below is one captured
+        # graph of R back-to-back launches, timed by one event pair and divided by R, so no
+        # launch or event floor enters it. The launches rotate over N_ROT score sets with
+        # different selections, so consecutive steps gather different blocks and K/V is read
+        # from HBM (only the current block, the same in every set, can stay in L2).
+        N_ROT, R = 4, 32
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(4242)
+        s_rot = [xd["s"]] + [torch.randn(xd["s"].shape, generator=gen, device=dev) * 2 ** 0.5
+                             for _ in range(N_ROT - 1)]
+        o_rot = [od] + [sas.empty_decode_outputs(pd, n_split, device=dev) for _ in range(N_ROT - 1)]
+        cl = xd["cache_len"]
+        with torch.cuda.stream(stream):
+            for k_ in range(N_ROT):  # each set's index lists and partials exist before any timing
+                sas.decode_step(pd, xd["q"], xd["k"], xd["v"], cl, s_rot[k_], n_split, o_rot[k_], stream=stream)
         kernels = {
-            "select": lambda: sas.sas_topk_select(pd, xd["s"], od["idx"], od["lse_s"], cache_len=xd["cache_len"],
-                                                  stream=stream),
-            "split": lambda: sas.sas_decode(pd, xd["q"], xd["k"], xd["v"], xd["cache_len"], xd["s"], od["idx"],
-                                            od["lse_s"], n_split, od["o_part"], od["lse_part"], stream=stream),
-            "combine": lambda: sas.sas_decode_combine(pd, n_split, od["o_part"], od["lse_part"], od["o"],
-                                                      od["lse_o"], stream=stream)}
+            "select": lambda k_: sas.sas_topk_select(pd, s_rot[k_], o_rot[k_]["idx"], o_rot[k_]["lse_s"],
+                                                     cache_len=cl, stream=stream),
+            "split": lambda k_: sas.sas_decode(pd, xd["q"], xd["k"], xd["v"], cl, s_rot[k_], o_rot[k_]["idx"],
+                                               o_rot[k_]["lse_s"], n_split, o_rot[k_]["o_part"],
+                                               o_rot[k_]["lse_part"], stream=stream),
+            "combine": lambda k_: sas.sas_decode_combine(pd, n_split, o_rot[k_]["o_part"], o_rot[k_]["lse_part"],
+                                                         o_rot[k_]["o"], o_rot[k_]["lse_o"], stream=stream),
+            "step": lambda k_: sas.decode_step(pd, xd["q"], xd["k"], xd["v"], cl, s_rot[k_], n_split, o_rot[k_],
+                                               stream=stream)}
+
+        def capture_r(fn):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+                for r_ in range(R):
+                    fn(r_ % N_ROT)
+            return g
+
+        graphs = {key: capture_r(fn) for key, fn in kernels.items()}
+        step_graph = sas.DecodeGraph(pd, xd["q"], xd["k"], xd["v"], cl, xd["s"], n_split, od, stream=stream)
 
         def replay_timed(g):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -459,55 +475,45 @@ def run_gpu(args, rank, world, local_rank):
             ev[1].record(stream)
             return ev
 
-        def eager_timed(fn):
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-            ev[0].record(stream)
-            fn()
-            ev[1].record(stream)
-            return ev
-
-        n_dec = max(20, args.steps * 4)
-        timings = {"step": [], "eager": [], "select": [], "split": [], "combine": []}
+        n_rep = max(5, args.steps // 2)
+        timings = {key: [] for key in graphs}
+        flushed = []
         with torch.cuda.stream(stream):
             for _ in range(max(3, args.warmup)):
+                for g in graphs.values():
+                    g.replay()
                 step_graph.replay()
-                dstep_eager()
-            for _ in range(n_dec):
-                for key, fn in (("step", lambda: replay_timed(step_graph.graph)), ("eager", dstep_eager),
-                                ("select", lambda: eager_timed(kernels["select"])),
-                                ("split", lambda: eager_timed(kernels["split"])),
-                                ("combine", lambda: eager_timed(kernels["combine"]))):
-                    torch.sum(flush, dim=0, out=flush_sink)
-                    timings[key].append(fn())
-            # a serving loop's view: R steps back to back (no flush), one event pair
-            r_hot = 50
-            hot = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-            hot[0].record(stream)
-            for _ in range(r_hot):
-                step_graph.replay()
-            hot[1].record(stream)
+            for _ in range(n_rep):
+                for key, g in graphs.items():
+                    timings[key].append(replay_timed(g))
+            # the conservative view: one step after an L2 flush (includes one graph launch)
+            for _ in range(max(20, args.steps)):
+                torch.sum(flush, dim=0, out=flush_sink)
+                flushed.append(replay_timed(step_graph.graph))
         torch.cuda.synchronize()
-        med = {key: statistics.median(e[0].elapsed_time(e[1]) for e in evs) for key, evs in timings.items()}
-        med["hot"] = hot[0].elapsed_time(hot[1]) / r_hot
+        med = {key: statistics.median(e[0].elapsed_time(e[1]) for e in evs) / R for key, evs in timings.items()}
+        med["flushed"] = statistics.median(e[0].elapsed_time(e[1]) for e in flushed)
         step_ms = max_over_ranks(dist, med["step"], dev)
         split_ms = med["split"]
         kv = decode_kv_bytes(wd, xd["cache_len"].cpu().numpy())
         gbs = kv / (split_ms * 1e-3) / 1e9
         line["decode"] = {
             "workload": DECODE, "tok_per_s": job_rate(wd.batch, world, step_ms * 1e-3), "ms_per_step": step_ms,
-            "launch": "CUDA graph of the three kernels, chained by programmatic dependent launch",
-            "eager_ms_per_step": med["eager"], "select_ms": med["select"], "split_ms": split_ms,
-            "combine_ms": med["combine"], "n_split": n_split,
-            "breakdown": "each kernel launched alone between two events after an L2 flush",
-            "hot_ms_per_step": med["hot"],
-            "hot": "50 graph replays back to back between one event pair, no flush (K/V partly in L2)",
-            "gate": "none (inference form)", "l2": "flushed (252 MB read) before every timed replay",
+            "launch": f"{R} steps back to back in one CUDA graph (three kernels each, chained by programmatic "
+                      f"dependent launch), rotating over {N_ROT} score sets with different selections",
+            "select_ms": med["select"], "split_ms": split_ms, "combine_ms": med["combine"], "n_split": n_split,
+            "breakdown": f"each kernel as {R} back-to-back launches in one graph over the rotating sets, / {R}",
+            "flushed_ms_per_step": med["flushed"],
+            "flushed": "one captured step replayed after a 252 MB read that flushes the L2 (one graph launch "
+                       "included)",
+            "gate": "none (inference form)",
+            "l2": "no flush: consecutive steps gather different blocks (rotating selections)",
             "roofline": {"bound": "hbm", "kernel": "decode_split_kernel (sas_decode)", "achieved": gbs,
                          "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"], "algorithmic_bytes": kv,
                          "traffic": traffic_record("decode_split",
                                                    ["learned_block_sparse_warp_b200/csrc/decode.cu"])},
             "gpu_launches_per_step": 3}
-        del step_graph, kernels
+        del step_graph, kernels, graphs, o_rot, s_rot
         if sas.sas_get_device_error(stream) != 0:
             raise RuntimeError("device error during decode")
         # the captured step at other split counts, for the choice of the default (the headline stays
@@ -644,6 +650,8 @@ def sweep_section(args, sas, stream, dev, pk, dist, world):
     from synth import workloads as W
     points = []
     for name in SWEEP:
+        if args.sweep_point and name != args.sweep_point:
+            continue
         w = W.WORKLOADS[name]
         p = sas.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
                        seq_len=w.seq_len, top_k=w.top_k, gate_mode=sas.SAS_GATE_LOG_SOFTMAX)
@@ -717,8 +725,6 @@ def long_decode_section(args, sas, stream, dev, pk, dist, world):
     import torch
     out_rows = []
     Hq, Hkv, d, K = 32, 8, 128, 16
-    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
 
     def timed(g):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -742,47 +748,60 @@ def long_decode_section(args, sas, stream, dev, pk, dist, world):
             sas.sas_block_mean_keys(p, kc, km, stream=stream)  # after the prefill: every block
             s = torch.empty((B, Hkv, NB), dtype=torch.float32, device=dev)
         n_split = K + 1
-        od = sas.empty_decode_outputs(p, n_split, device=dev)
-        step = sas.DecodeGraph(p, q, kc, vc, cl, s, n_split, od, stream=stream, kmean=km)
+        # N_ROT query sets with their own outputs: consecutive steps select different blocks
+        N_ROT, R = 4, 32
+        q_rot = [q] + [torch.randn((B, Hq, d), generator=gen, device=dev, dtype=torch.bfloat16)
+                       for _ in range(N_ROT - 1)]
+        s_rot = [s] + [torch.empty_like(s) for _ in range(N_ROT - 1)]
+        o_rot = [sas.empty_decode_outputs(p, n_split, device=dev) for _ in range(N_ROT)]
+        with torch.cuda.stream(stream):
+            for k_ in range(N_ROT):
+                sas.decode_step_scored(p, q_rot[k_], kc, vc, km, cl, s_rot[k_], n_split, o_rot[k_], stream=stream)
         kernels = {
-            "mean_update": lambda: sas.sas_block_mean_keys(p, kc, km, cache_len=cl, stream=stream),
-            "select": lambda: sas.sas_decode_select_scored(p, q, km, cl, s, od["idx"], od["lse_s"], stream=stream),
-            "split": lambda: sas.sas_decode(p, q, kc, vc, cl, s, od["idx"], od["lse_s"], n_split, od["o_part"],
-                                            od["lse_part"], stream=stream),
-            "combine": lambda: sas.sas_decode_combine(p, n_split, od["o_part"], od["lse_part"], od["o"],
-                                                      od["lse_o"], stream=stream)}
+            "mean_update": lambda k_: sas.sas_block_mean_keys(p, kc, km, cache_len=cl, stream=stream),
+            "select": lambda k_: sas.sas_decode_select_scored(p, q_rot[k_], km, cl, s_rot[k_], o_rot[k_]["idx"],
+                                                              o_rot[k_]["lse_s"], stream=stream),
+            "split": lambda k_: sas.sas_decode(p, q_rot[k_], kc, vc, cl, s_rot[k_], o_rot[k_]["idx"],
+                                               o_rot[k_]["lse_s"], n_split, o_rot[k_]["o_part"],
+                                               o_rot[k_]["lse_part"], stream=stream),
+            "combine": lambda k_: sas.sas_decode_combine(p, n_split, o_rot[k_]["o_part"], o_rot[k_]["lse_part"],
+                                                         o_rot[k_]["o"], o_rot[k_]["lse_o"], stream=stream),
+            "step": lambda k_: sas.decode_step_scored(p, q_rot[k_], kc, vc, km, cl, s_rot[k_], n_split, o_rot[k_],
+                                                      stream=stream)}
         # unfused comparison: the scores by a library batched matmul, then the separate Top-K kernel
         qbar = torch.empty((B * Hkv, d, 1), dtype=torch.bfloat16, device=dev)
         s_mm = torch.empty((B * Hkv, NB, 1), dtype=torch.bfloat16, device=dev)
         s_un = torch.empty((B, Hkv, NB), dtype=torch.float32, device=dev)
 
-        def unfused():
-            qbar.copy_(q.view(B * Hkv, Hq // Hkv, d).float().mean(dim=1).mul_(d ** -0.5).unsqueeze(-1))
+        def unfused(k_):
+            qbar.copy_(q_rot[k_].view(B * Hkv, Hq // Hkv, d).float().mean(dim=1).mul_(d ** -0.5).unsqueeze(-1))
             torch.bmm(km.view(B * Hkv, NB, d), qbar, out=s_mm)
             s_un.view(B * Hkv, NB).copy_(s_mm.view(B * Hkv, NB))
-            sas.sas_topk_select(p, s_un, od["idx"], od["lse_s"], cache_len=cl, stream=stream)
+            sas.sas_topk_select(p, s_un, o_rot[k_]["idx"], o_rot[k_]["lse_s"], cache_len=cl, stream=stream)
 
+        with torch.cuda.stream(stream):
+            unfused(0)  # first call outside capture: the library GEMM's handle is created here
         kernels["select_unfused"] = unfused
-        # the step is the captured graph a serving loop replays; each kernel is launched alone between
-        # two events, queued behind the L2 flush, so the event pair spans the kernel only
-        times = {k: [] for k in ["step", *kernels]}
+
+        # each figure: one graph of R back-to-back launches over the rotating sets, / R
+        def capture_r(fn):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+                for r_ in range(R):
+                    fn(r_ % N_ROT)
+            return g
+
+        graphs = {key: capture_r(fn) for key, fn in kernels.items()}
+        times = {k: [] for k in graphs}
         with torch.cuda.stream(stream):
             for _ in range(max(3, args.warmup)):
-                step.graph.replay()
-                for fn in kernels.values():
-                    fn()
-            for _ in range(max(10, args.steps)):
-                torch.sum(flush, dim=0, out=flush_sink)
-                times["step"].append(timed(step.graph))
-                for key, fn in kernels.items():
-                    torch.sum(flush, dim=0, out=flush_sink)
-                    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-                    ev[0].record(stream)
-                    fn()
-                    ev[1].record(stream)
-                    times[key].append(ev)
+                for g in graphs.values():
+                    g.replay()
+            for _ in range(max(5, args.steps // 2)):
+                for key, g in graphs.items():
+                    times[key].append(timed(g))
         torch.cuda.synchronize()
-        med = {k: statistics.median(e[0].elapsed_time(e[1]) for e in evs) for k, evs in times.items()}
+        med = {k: statistics.median(e[0].elapsed_time(e[1]) for e in evs) / R for k, evs in times.items()}
         if sas.sas_get_device_error(stream) != 0:
             raise RuntimeError("device error during long-context decode")
         step_ms = max_over_ranks(dist, med["step"], dev)
@@ -798,12 +817,14 @@ def long_decode_section(args, sas, stream, dev, pk, dist, world):
             "select_roofline": {"bound": "hbm", "kernel": "select_scored_kernel (sas_decode_select_scored)",
                                 "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
                                 "algorithmic_bytes": sel_bytes}})
-        del step, kernels, kc, vc, km, s, od
+        del kernels, graphs, kc, vc, km, s, s_rot, q_rot, o_rot
         torch.cuda.empty_cache()
     return {"workloads": out_rows, "gate": "none (inference form)", "n_split": K + 1,
             "data": "synthetic: q, k, v ~ N(0, 1) bf16 from a seeded device generator",
-            "launch": "one CUDA graph per step: block-mean update, fused scoring + Top-K, split-K, merge (PDL-chained)",
-            "l2": "flushed (252 MB read) before every timed replay", "gpu_launches_per_step": 4}
+            "launch": "steps of four PDL-chained kernels (block-mean update, fused scoring + Top-K, split-K, merge); "
+                      "every figure is one graph of 32 back-to-back launches / 32",
+            "l2": "no flush: the launches rotate over 4 query sets, so consecutive steps select different blocks",
+            "gpu_launches_per_step": 4}
 
 
 # ---------------------------------------------------------------------------
@@ -843,6 +864,7 @@ def main():
     ap.add_argument("--only", choices=["all", "train", "decode", "long_decode", "sweep"], default="all",
                     help="run only one workload (for profiling); the JSON line needs 'all'")
     ap.add_argument("--n-split", type=int, default=0, help="decode splits (0: K + 1)")
+    ap.add_argument("--sweep-point", default="", help="with --only sweep: run this sweep workload alone (profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -935,12 +935,12 @@ __global__ void __launch_bounds__(bdq::kThreads, 2)
         if (!(ok = mbar_wait(smem_u32(&bar_full[st]), use & 1, abort_flag, a.err))) break;
         tc_fence_after();
         const uint32_t so = st * bdq::kStage;
-        for (int r = 0; r < n_tiles; ++r) {
+        // K steps outer, tiles inner: consecutive MMAs feed different accumulators
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < 4; ++k)
+          for (int r = 0; r < n_tiles; ++r)
             mma_ss(tmem + r * 128, desc_advance(dZ0, so + r * bdq::kTileZ + k * 32), desc_advance(dK0, so + k * 2048),
                    idQ, (i > 0 || k > 0) ? 1u : 0u);
-        }
         mma_commit(smem_u32(&bar_empty[st]));
       }
       mma_commit(smem_u32(&bar_fin));
