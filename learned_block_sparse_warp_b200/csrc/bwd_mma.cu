@@ -1,4 +1,5 @@
-// Backward of gated block-sparse attention, with the gate/score gradient.
+// Backward of gated block-sparse attention: the small kernels around the
+// tcgen05 passes, the workspace layout, and the launcher.
 //
 // SAS summary (onedev.kr), section 무엇과 다른가: with the gate inside the
 // softmax the gate gradient is dg_m = Σ_i (p̃_i/g_m) dOᵀ(v_i − o), and
@@ -16,16 +17,9 @@
 //   revidx_count/scan/fill
 //                    for every KV block j, the query blocks t > j that
 //                    selected it, ascending in t, with j's slot in idx[t]
-//   bwd_main         one CTA per (batch, KV head, KV block j), eight warps.
-//                    It walks its diagonal query block and then every query
-//                    block that selected j, for each of the G heads, and
-//                    recomputes P from the saved row LSE. dK_j and dV_j stay
-//                    in registers for the whole walk. dQ is added to an fp32
-//                    workspace with red.global. dl[t, slot] has exactly one
-//                    writer, the CTA that owns j, so the score path uses no
-//                    atomics.
-//   bwd_dq_convert   fp32 dQ -> bf16
-//   bwd_ds_chain     ds from dl through the softmax over s
+//                    and the block's log2 gate for t
+//   the tcgen05 passes (bwd_sm100.cu): dK, dV, dl (and the dZ tiles), then dQ
+//   bwd_ds_chain     ds from dl through the gate's activation
 #include <algorithm>
 
 #include "common.cuh"
@@ -33,14 +27,13 @@
 namespace sas {
 
 struct BwdWs {
-  float* dq_acc;   // [B, Hq, N, d] fp32 (d = 64 path only)
   float* drow;     // [B, Hq, N]
   float* dl;       // [B, Hkv, NB, K]
   int* rev_cnt;    // [B, Hkv, NB]
   int* rev_off;    // [B, Hkv, NB + 1]
   int* rev_list;   // [B, Hkv, NB * K]: (t << kSlotBits) | slot
   float* rev_lam;  // [B, Hkv, NB * K]: log2-domain gate of each reverse-index entry
-  uint16_t* dz;    // d = 128 with spill: [B, Hkv, Σ_t (1 + min(K, t)), ceil(G/2)] tiles of 128 x 64 bf16
+  uint16_t* dz;    // with spill: [B, Hkv, Σ_t (1 + min(K, t)), ceil(G/2)] tiles of 128 x 64 bf16
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -49,13 +42,11 @@ long long bwd_dz_tiles(const Shape& sh);
 
 // The stored-dZ backward needs one 16 KB tile per (query block, attended block,
 // head pair); its tile index must fit a TMA coordinate.
-bool bwd_can_spill(const Shape& sh) { return sh.d == 128 && bwd_dz_tiles(sh) < (1LL << 31); }
+bool bwd_can_spill(const Shape& sh) { return bwd_dz_tiles(sh) < (1LL << 31); }
 
 size_t bwd_ws_layout(const Shape& sh, bool spill, void* base, BwdWs* ws) {
   const size_t bhq = size_t(sh.B) * sh.Hq, bhk = size_t(sh.B) * sh.Hkv;
   size_t off = 0;
-  size_t o_dq = off;
-  if (sh.d != 128) off = align256(off + bhq * sh.N * sh.d * sizeof(float));
   size_t o_dr = off;
   off = align256(off + bhq * sh.N * sizeof(float));
   size_t o_dl = off;
@@ -72,7 +63,6 @@ size_t bwd_ws_layout(const Shape& sh, bool spill, void* base, BwdWs* ws) {
   if (spill) off = align256(off + size_t(bwd_dz_tiles(sh)) * 128 * 64 * sizeof(uint16_t));
   if (ws != nullptr) {
     char* p = static_cast<char*>(base);
-    ws->dq_acc = sh.d != 128 ? reinterpret_cast<float*>(p + o_dq) : nullptr;
     ws->drow = reinterpret_cast<float*>(p + o_dr);
     ws->dl = reinterpret_cast<float*>(p + o_dl);
     ws->rev_cnt = reinterpret_cast<int*>(p + o_cnt);
@@ -205,259 +195,6 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const int32_t* __restr
   }
 }
 
-// ---------------------------------------------------------------------------
-// Main backward kernel
-// ---------------------------------------------------------------------------
-template <int D>
-__device__ __forceinline__ void bwd_load_tile(uint32_t s_base, const uint16_t* __restrict__ g, int tid) {
-  constexpr int CH = D / 8;
-  for (int i = tid; i < kBlock * CH; i += 256) {
-    const int r = i / CH, c = i % CH;
-    cp_async16(s_base + swz<CH>(r, c), g + size_t(r) * D + c * 8);
-  }
-}
-
-__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(addr), "r"(v));
-}
-
-__device__ __forceinline__ void red_add_f32x2(float* p, float a, float b) {
-  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};\n" ::"l"(p), "f"(a), "f"(b) : "memory");
-}
-
-template <int D>
-__global__ void __launch_bounds__(256, 1) bwd_main_kernel(
-    const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-    const uint16_t* __restrict__ dO, const float* __restrict__ s, const float* __restrict__ lse_s,
-    const float* __restrict__ lse_o, const float* __restrict__ drow, const int* __restrict__ rev_off,
-    const int* __restrict__ rev_list, float* __restrict__ dq_acc, float* __restrict__ dl, uint16_t* __restrict__ dk,
-    uint16_t* __restrict__ dv, Shape sh) {
-  constexpr int CH = D / 8;
-  constexpr int TILE = kBlock * D * 2;
-  constexpr int PT = kBlock * kBlock * 2;  // 64 x 64 bf16
-  constexpr int NT = D / 16;               // 8-wide d tiles per warp (half of D)
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(16) float sL[2][kBlock];
-  __shared__ __align__(16) float sD[2][kBlock];
-  __shared__ float sdl[8];
-
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const size_t bh = size_t(b) * sh.Hkv + h;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wm = warp & 3, wn = warp >> 2;
-  const uint32_t sK = smem_u32(smem);
-  const uint32_t sV = sK + TILE;
-  const uint32_t sQ = sV + TILE;       // 2 stages
-  const uint32_t sdO = sQ + 2 * TILE;  // 2 stages
-  const uint32_t sP = sdO + 2 * TILE;
-  const uint32_t sZ = sP + PT;
-  const int G = sh.G;
-
-  const int off0 = rev_off[bh * (sh.NB + 1) + j];
-  const int n_sel = rev_off[bh * (sh.NB + 1) + j + 1] - off0;
-  const int* lst = rev_list + bh * size_t(sh.NB) * sh.K + off0;
-  const int n_steps = (1 + n_sel) * G;
-
-  auto step_t = [&](int e) -> int { return e == 0 ? j : (lst[e - 1] >> kSlotBits); };
-  auto issue_step = [&](int st, int stage) {
-    const int e = st / G, g = st % G;
-    const int t = step_t(e);
-    const int hq = h * G + g;
-    const size_t rowbase = (size_t(b) * sh.Hq + hq) * sh.N + size_t(t) * kBlock;
-    bwd_load_tile<D>(sQ + stage * TILE, q + rowbase * D, tid);
-    bwd_load_tile<D>(sdO + stage * TILE, dO + rowbase * D, tid);
-    if (tid < 16) cp_async16(smem_u32(&sL[stage][tid * 4]), lse_o + rowbase + tid * 4);
-    else if (tid < 32) cp_async16(smem_u32(&sD[stage][(tid - 16) * 4]), drow + rowbase + (tid - 16) * 4);
-  };
-
-  const uint16_t* kg = k + (bh * sh.N + size_t(j) * kBlock) * D;
-  const uint16_t* vg = v + (bh * sh.N + size_t(j) * kBlock) * D;
-  bwd_load_tile<D>(sK, kg, tid);
-  bwd_load_tile<D>(sV, vg, tid);
-  issue_step(0, 0);
-  cp_async_commit();
-
-  float dk_acc[NT][4], dv_acc[NT][4];
-#pragma unroll
-  for (int i = 0; i < NT; ++i)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dk_acc[i][e] = dv_acc[i][e] = 0.f;
-  float dl_part = 0.f;
-  const float sc2 = sh.scale * kLog2e;
-  const int ra = 16 * wm + (lane >> 2);  // this thread's S rows: ra, ra + 8
-  const int ca = 32 * wn;                // this warp's S columns: ca .. ca + 31
-
-  for (int st = 0; st < n_steps; ++st) {
-    const int stage = st & 1;
-    if (st + 1 < n_steps) {
-      issue_step(st + 1, stage ^ 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int e = st / G, g = st % G;
-    const int t = step_t(e);
-    const int slot = e == 0 ? -1 : (lst[e - 1] & ((1 << kSlotBits) - 1));
-    const bool diag = (e == 0);
-    float lam2 = 0.f;
-    if (!diag && sh.gated) {
-      const size_t row = bh * sh.NB + t;
-      lam2 = gate_lam2(sh.gate, s[row * sh.NB + j], lse_s != nullptr ? lse_s[row] : 0.f);
-    }
-    const uint32_t cQ = sQ + stage * TILE, cdO = sdO + stage * TILE;
-    // Gate inside the softmax: log2 g biases the logits. Outside: the logits are
-    // plain, v carries the weight g·p, so dV takes g·p, dZ = p·(g·dP − D), and
-    // dl = Σ p·g·dP (= g ∂/∂g).
-    const float zb = sh.outside ? 0.f : lam2;
-    const float gw = sh.outside ? exp2f(lam2) : 1.f;
-
-    // S = Q Kᵀ and dP = dO Vᵀ for rows 16wm.., columns 32wn..
-    float sacc[4][4], pacc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) sacc[i][c] = pacc[i][c] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t a[4], ad[4];
-      ldsm_x4(cQ + swz<CH>(16 * wm + (lane & 15), 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
-      ldsm_x4(cdO + swz<CH>(16 * wm + (lane & 15), 2 * kk + (lane >> 4)), ad[0], ad[1], ad[2], ad[3]);
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        const int brow = ca + 16 * np + (lane & 7) + ((lane >> 4) << 3);
-        const int bch = 2 * kk + ((lane >> 3) & 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(sK + swz<CH>(brow, bch), b0, b1, b2, b3);
-        mma_bf16_16816(sacc[2 * np], a, b0, b1);
-        mma_bf16_16816(sacc[2 * np + 1], a, b2, b3);
-        ldsm_x4(sV + swz<CH>(brow, bch), b0, b1, b2, b3);
-        mma_bf16_16816(pacc[2 * np], ad, b0, b1);
-        mma_bf16_16816(pacc[2 * np + 1], ad, b2, b3);
-      }
-    }
-    // P and dZ, stored to shared memory as bf16; dl partial sum in fp32
-    {
-      const float L0 = sL[stage][ra] * kLog2e, L1 = sL[stage][ra + 8] * kLog2e;
-      const float D0 = sD[stage][ra], D1 = sD[stage][ra + 8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int col = ca + 8 * i + 2 * (lane & 3);
-        float p[4], z[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int row = ra + ((c >> 1) << 3);
-          const int cc = col + (c & 1);
-          const float Lr = (c >> 1) ? L1 : L0;
-          const float Dr = (c >> 1) ? D1 : D0;
-          float pv = exp2f(fmaf(sacc[i][c], sc2, zb) - Lr);
-          if (diag && cc > row) pv = 0.f;
-          const float gdp = gw * pacc[i][c];
-          p[c] = pv * gw;
-          z[c] = pv * (gdp - Dr);
-          dl_part += sh.outside ? pv * gdp : z[c];
-        }
-        st_shared_b32(sP + swz<8>(ra, col >> 3) + (col & 7) * 2, pack_bf16x2(p[0], p[1]));
-        st_shared_b32(sP + swz<8>(ra + 8, col >> 3) + (col & 7) * 2, pack_bf16x2(p[2], p[3]));
-        st_shared_b32(sZ + swz<8>(ra, col >> 3) + (col & 7) * 2, pack_bf16x2(z[0], z[1]));
-        st_shared_b32(sZ + swz<8>(ra + 8, col >> 3) + (col & 7) * 2, pack_bf16x2(z[2], z[3]));
-      }
-    }
-    const bool last_head = (g == G - 1);
-    if (last_head && !diag) {
-      const float w = warp_sum(dl_part);
-      if (lane == 0) sdl[warp] = w;
-    }
-    __syncthreads();
-
-    // dV += Pᵀ dO and dK += dZᵀ Q: rows = KV tokens 16wm.., cols = d (D/2)wn..
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t ap[4], az[4];
-      const int arow = 16 * kk + (lane & 7) + ((lane >> 4) << 3);
-      const int ach = 2 * wm + ((lane >> 3) & 1);
-      ldsm_x4_t(sP + swz<8>(arow, ach), ap[0], ap[1], ap[2], ap[3]);
-      ldsm_x4_t(sZ + swz<8>(arow, ach), az[0], az[1], az[2], az[3]);
-#pragma unroll
-      for (int dp = 0; dp < NT / 2; ++dp) {
-        const int brow = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
-        const int bch = (D / 16) * wn + 2 * dp + (lane >> 4);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(cdO + swz<CH>(brow, bch), b0, b1, b2, b3);
-        mma_bf16_16816(dv_acc[2 * dp], ap, b0, b1);
-        mma_bf16_16816(dv_acc[2 * dp + 1], ap, b2, b3);
-        ldsm_x4_t(cQ + swz<CH>(brow, bch), b0, b1, b2, b3);
-        mma_bf16_16816(dk_acc[2 * dp], az, b0, b1);
-        mma_bf16_16816(dk_acc[2 * dp + 1], az, b2, b3);
-      }
-    }
-    // dQ = scale · dZ K: rows = queries 16wm.., cols = d (D/2)wn..
-    {
-      float qacc[NT][4];
-#pragma unroll
-      for (int i = 0; i < NT; ++i) qacc[i][0] = qacc[i][1] = qacc[i][2] = qacc[i][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t a[4];
-        ldsm_x4(sZ + swz<8>(16 * wm + (lane & 15), 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
-#pragma unroll
-        for (int dp = 0; dp < NT / 2; ++dp) {
-          const int brow = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
-          const int bch = (D / 16) * wn + 2 * dp + (lane >> 4);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sK + swz<CH>(brow, bch), b0, b1, b2, b3);
-          mma_bf16_16816(qacc[2 * dp], a, b0, b1);
-          mma_bf16_16816(qacc[2 * dp + 1], a, b2, b3);
-        }
-      }
-      const int hq = h * G + g;
-      float* dqb = dq_acc + ((size_t(b) * sh.Hq + hq) * sh.N + size_t(t) * kBlock) * D;
-#pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        const int col = (D / 2) * wn + 8 * i + 2 * (lane & 3);
-        red_add_f32x2(dqb + size_t(ra) * D + col, qacc[i][0] * sh.scale, qacc[i][1] * sh.scale);
-        red_add_f32x2(dqb + size_t(ra + 8) * D + col, qacc[i][2] * sh.scale, qacc[i][3] * sh.scale);
-      }
-    }
-    __syncthreads();
-    if (last_head) {
-      if (!diag && sh.gated && tid == 0) {
-        float w = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) w += sdl[i];
-        dl[(bh * sh.NB + t) * sh.K + slot] = w;
-      }
-      dl_part = 0.f;
-    }
-  }
-
-  // dK (scaled) and dV of block j, summed over the G heads
-  uint16_t* dkg = dk + (bh * sh.N + size_t(j) * kBlock) * D;
-  uint16_t* dvg = dv + (bh * sh.N + size_t(j) * kBlock) * D;
-#pragma unroll
-  for (int i = 0; i < NT; ++i) {
-    const int col = (D / 2) * wn + 8 * i + 2 * (lane & 3);
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = ra + 8 * r;
-      *reinterpret_cast<uint32_t*>(dkg + size_t(row) * D + col) =
-          pack_bf16x2(dk_acc[i][2 * r] * sh.scale, dk_acc[i][2 * r + 1] * sh.scale);
-      *reinterpret_cast<uint32_t*>(dvg + size_t(row) * D + col) = pack_bf16x2(dv_acc[i][2 * r], dv_acc[i][2 * r + 1]);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Epilogues
-// ---------------------------------------------------------------------------
-__global__ void bwd_dq_convert_kernel(const float4* __restrict__ acc, size_t n4, uint2* __restrict__ out) {
-  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += size_t(gridDim.x) * blockDim.x) {
-    const float4 a = acc[i];
-    out[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
-  }
-}
-
 // One warp per (b, h, t): ds[t, m] = dl[t, m]·[m∈I] − softmax(s_t)_m Σ dl.
 __global__ void __launch_bounds__(256) bwd_ds_chain_kernel(const float* __restrict__ s, const float* __restrict__ lse_s,
                                                            const int32_t* __restrict__ idx,
@@ -529,27 +266,11 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
   revidx_count_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_cnt);
   revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
   revidx_fill_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_off, ws.rev_list, s, lse_s,
-                                                    sh.gate, D == 128 ? ws.rev_lam : nullptr);
-  if (D == 128) {  // tcgen05 passes: dK/dV/dl (and the dZ tiles) KV-major, then dQ query-major
-    if ((e = launch_bwd_passes_sm100(sh, q, k, v, dO, s, idx, lse_s, lse_o, ws.drow, ws.rev_off, ws.rev_list,
-                                     ws.rev_lam, ws.dl, ws.dz, dq, dk, dv, err, st)) != cudaSuccess)
-      return e;
-    if (ds != nullptr) {
-      const int rows = nbh * sh.NB;
-      bwd_ds_chain_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, lse_s, idx, ws.dl, rows, sh.NB, sh.K, sh.gate, ds);
-    }
-    return cudaGetLastError();
-  }
-  if ((e = cudaMemsetAsync(ws.dq_acc, 0, rows_q * D * sizeof(float), st)) != cudaSuccess) return e;
-  const int smem = 6 * kBlock * D * 2 + 2 * kBlock * kBlock * 2;
-  if ((e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
-      cudaSuccess)
+                                                    sh.gate, ws.rev_lam);
+  // tcgen05 passes: dK/dV/dl (and the dZ tiles) KV-major, then dQ query-major
+  if ((e = launch_bwd_passes_sm100(sh, q, k, v, dO, s, idx, lse_s, lse_o, ws.drow, ws.rev_off, ws.rev_list,
+                                   ws.rev_lam, ws.dl, ws.dz, dq, dk, dv, err, st)) != cudaSuccess)
     return e;
-  bwd_main_kernel<D><<<dim3(sh.NB, sh.Hkv, sh.B), 256, smem, st>>>(q, k, v, dO, s, lse_s, lse_o, ws.drow, ws.rev_off,
-                                                                   ws.rev_list, ws.dq_acc, ws.dl, dk, dv, sh);
-  const size_t n4 = rows_q * D / 4;
-  bwd_dq_convert_kernel<<<148 * 8, 256, 0, st>>>(reinterpret_cast<const float4*>(ws.dq_acc), n4,
-                                                  reinterpret_cast<uint2*>(dq));
   if (ds != nullptr) {
     const int rows = nbh * sh.NB;
     bwd_ds_chain_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, lse_s, idx, ws.dl, rows, sh.NB, sh.K, sh.gate, ds);
@@ -563,7 +284,7 @@ cudaError_t launch_bwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k
                            void* ws, bool spill, int* err, cudaStream_t st) {
   if (sh.d == 128)
     return launch_bwd_d<128>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, spill, err, st);
-  return launch_bwd_d<64>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, false, err, st);
+  return launch_bwd_d<64>(sh, q, k, v, o, dO, s, idx, lse_s, lse_o, dq, dk, dv, ds, ws, spill, err, st);
 }
 
 }  // namespace sas

@@ -43,6 +43,7 @@ struct BwdSm100Args {
   const int32_t* idx;
   int* err;
   int B, Hq, Hkv, G, N, NB, K, gate, gated, n_hp, n_tp;
+  int d;  // head dim, 64 or 128; at 64 the tensor maps zero-fill the second 64-column half of every box
   float scale;
   int spill;            // 1: the KV pass stores every dZ tile and the dQ pass reads them back
   long long dz_slots;   // dZ slots per (batch, KV head): Σ_t (1 + min(K, t))
@@ -514,13 +515,14 @@ __global__ void __launch_bounds__(bkv::kThreads, 1)
       }
     }
     named_bar_sync(2 + (is_v ? 0 : 1), 256);
-    if (ok) {
-      uint16_t* dst = (is_v ? a.dv : a.dk) + (bh * a.N + size_t(j) * kBlock) * 128;
+    if (ok) {  // the staged rows hold 128 d; the first d of them go out
+      const int cpr = a.d / 8;  // 16-byte chunks per output row
+      uint16_t* dst = (is_v ? a.dv : a.dk) + (bh * a.N + size_t(j) * kBlock) * a.d;
       uint4* g = reinterpret_cast<uint4*>(dst);
-      for (int i = (cg & 1) * 128 + row; i < 64 * 16; i += 256) {
+      for (int i = (cg & 1) * 128 + row; i < 64 * cpr; i += 256) {
         uint4 x;
         asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
-                     : "r"(stage_buf + i * 16));
+                     : "r"(stage_buf + ((i / cpr) * 16 + i % cpr) * 16));
         g[i] = x;
       }
     }
@@ -719,12 +721,13 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
     const size_t grow = (size_t(b) * a.Hq + (valid ? hq : h * a.G)) * a.N + size_t(t) * kBlock + qpos;
     {  // this thread's quarter of its row of Q and dO (d [32 cg, 32 cg + 32)) into TMEM; zero for a missing head
       uint32_t qw[16], ow[16];
-      const uint4* qg = reinterpret_cast<const uint4*>(q + grow * 128 + cg * 32);
-      const uint4* og = reinterpret_cast<const uint4*>(dO + grow * 128 + cg * 32);
+      const bool in_d = valid && cg * 32 < a.d;  // at d = 64 the upper half of the row is zero
+      const uint4* qg = reinterpret_cast<const uint4*>(q + grow * a.d + (in_d ? cg * 32 : 0));
+      const uint4* og = reinterpret_cast<const uint4*>(dO + grow * a.d + (in_d ? cg * 32 : 0));
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const uint4 x = valid ? qg[c] : make_uint4(0, 0, 0, 0);
-        const uint4 y = valid ? og[c] : make_uint4(0, 0, 0, 0);
+        const uint4 x = in_d ? qg[c] : make_uint4(0, 0, 0, 0);
+        const uint4 y = in_d ? og[c] : make_uint4(0, 0, 0, 0);
         qw[4 * c] = x.x, qw[4 * c + 1] = x.y, qw[4 * c + 2] = x.z, qw[4 * c + 3] = x.w;
         ow[4 * c] = y.x, ow[4 * c + 1] = y.y, ow[4 * c + 2] = y.z, ow[4 * c + 3] = y.w;
       }
@@ -780,12 +783,12 @@ __global__ void __launch_bounds__(bq::kThreads, 1)
     }
     if (ok) ok = mbar_wait(smem_u32(&bar_fin), 0, abort_flag, a.err);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && valid) {  // rows 64..127 of a one-head tile form whole warps
+    if (ok && valid && cg * 32 < a.d) {  // rows 64..127 of a one-head tile form whole warps
       tc_fence_after();
       uint32_t v[32];
       tmem_ld32(tmem + lane_addr + 256 + cg * 32, v);  // d columns [32 cg, 32 cg + 32)
       tmem_wait_ld();
-      uint4* og = reinterpret_cast<uint4*>(a.dq + grow * 128 + cg * 32);
+      uint4* og = reinterpret_cast<uint4*>(a.dq + grow * a.d + cg * 32);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint4 o4;
@@ -958,12 +961,12 @@ __global__ void __launch_bounds__(bdq::kThreads, 2)
         const int g = 2 * (hp0 + r) + (row >> 6);
         const bool valid = g < a.G;  // uniform over the warp: 32 rows of one head
         const size_t grow = (size_t(b) * a.Hq + size_t(h) * a.G + (valid ? g : 0)) * a.N + size_t(t) * kBlock + (row & 63);
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < a.d / 32; ++ch) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_addr + r * 128 + ch * 32, v);
           tmem_wait_ld();
           if (valid) {
-            uint4* og = reinterpret_cast<uint4*>(a.dq + grow * 128 + ch * 32);
+            uint4* og = reinterpret_cast<uint4*>(a.dq + grow * a.d + ch * 32);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               uint4 o4;
@@ -1007,8 +1010,10 @@ cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const ui
                                    uint16_t* dv, int* err, cudaStream_t st) {
   CUtensorMap tk, tv, tq3, tdo3, tl, td, tdz;
   const uint64_t hq = uint64_t(sh.B) * sh.Hq, rkv = uint64_t(sh.B) * sh.Hkv * sh.N;
-  if (!make_tmap_bf16_2d(&tk, k, rkv, 128) || !make_tmap_bf16_2d(&tv, v, rkv, 128) ||
-      !make_tmap_bf16_3d_heads(&tq3, q, hq, sh.N) || !make_tmap_bf16_3d_heads(&tdo3, dO, hq, sh.N) ||
+  // rows of d = 64 or 128 values: the kernels always load two 64-column boxes; at d = 64 the second
+  // lies past the extent and TMA fills it with zeros, which add nothing to any product
+  if (!make_tmap_bf16_2d(&tk, k, rkv, sh.d) || !make_tmap_bf16_2d(&tv, v, rkv, sh.d) ||
+      !make_tmap_bf16_3d_heads(&tq3, q, hq, sh.N, sh.d) || !make_tmap_bf16_3d_heads(&tdo3, dO, hq, sh.N, sh.d) ||
       !make_tmap_f32_rows(&tl, lse_o, hq, sh.N) || !make_tmap_f32_rows(&td, drow, hq, sh.N))
     return cudaErrorInvalidValue;
   // without a spill region the map is never used; it is encoded over the K cache so that it is valid
@@ -1040,6 +1045,7 @@ cudaError_t launch_bwd_passes_sm100(const Shape& sh, const uint16_t* q, const ui
   a.gated = sh.gated;
   a.n_hp = (sh.G + 1) / 2;
   a.n_tp = (sh.G + 3) / 4;
+  a.d = sh.d;
   a.scale = sh.scale;
   a.spill = dz != nullptr ? 1 : 0;
   a.dz_slots = dz_slot_base(sh.NB, sh.K);

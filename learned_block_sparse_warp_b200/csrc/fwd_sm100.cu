@@ -54,6 +54,7 @@ struct FwdSm100Args {
   float* lse_o;
   int* err;
   int B, Hq, Hkv, G, N, NB, K, gate, gated, n_tp;
+  int d;  // head dim, 64 or 128; at 64 the tensor maps zero-fill the second 64-column half of every box
   float scale;
 };
 
@@ -307,8 +308,8 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         const int hq = h * a.G + g_first + 2 * r + hh;
         const size_t orow = (size_t(b) * a.Hq + hq) * a.N + size_t(t) * kBlock + qpos;
         const float inv = 1.f / l;
-        uint4* og = reinterpret_cast<uint4*>(a.o + orow * 128);
-        for (int ch = 0; ch < 4; ++ch) {
+        uint4* og = reinterpret_cast<uint4*>(a.o + orow * a.d);
+        for (int ch = 0; ch < a.d / 32; ++ch) {
           uint32_t w[32];
           tmem_ld32(tO + ch * 32, w);
           tmem_wait_ld();
@@ -375,13 +376,14 @@ bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [heads, N, 128] read in boxes of 2 heads x 64 tokens x 64 d (128-byte swizzle), so one
-// load brings both heads of a head pair for one d-half: 128 rows of 128 B.
-bool make_tmap_bf16_3d_heads(CUtensorMap* m, const void* base, uint64_t heads, uint64_t N) {
+// bf16 [heads, N, d] read in boxes of 2 heads x 64 tokens x 64 d (128-byte swizzle), so one
+// load brings both heads of a head pair for one d-half: 128 rows of 128 B. At d = 64 the
+// second d-half is past the extent and arrives as zeros.
+bool make_tmap_bf16_3d_heads(CUtensorMap* m, const void* base, uint64_t heads, uint64_t N, uint64_t d) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return false;
-  const cuuint64_t dims[3] = {128, N, heads};
-  const cuuint64_t strides[2] = {128 * 2, N * 128 * 2};
+  const cuuint64_t dims[3] = {d, N, heads};
+  const cuuint64_t strides[2] = {d * 2, N * d * 2};
   const cuuint32_t box[3] = {64, 64, 2};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -420,8 +422,10 @@ cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t*
                              int* err, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   const uint64_t rq = uint64_t(sh.B) * sh.Hq * sh.N, rkv = uint64_t(sh.B) * sh.Hkv * sh.N;
-  if (!make_tmap_bf16_2d(&tq, q, rq, 128) || !make_tmap_bf16_2d(&tk, k, rkv, 128) ||
-      !make_tmap_bf16_2d(&tv, v, rkv, 128))
+  // [rows, d] with d = 64 or 128: the kernel always loads two 64-column boxes per row; at d = 64 the
+  // second lies past the extent, so TMA fills it with zeros and it adds nothing to S or to PV
+  if (!make_tmap_bf16_2d(&tq, q, rq, sh.d) || !make_tmap_bf16_2d(&tk, k, rkv, sh.d) ||
+      !make_tmap_bf16_2d(&tv, v, rkv, sh.d))
     return cudaErrorInvalidValue;
   auto kern = sh.outside ? fwd_sm100_kernel<true> : fwd_sm100_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fsm::kSmemBytes);
@@ -443,6 +447,7 @@ cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t*
   a.gate = sh.gate;
   a.gated = sh.gated;
   a.n_tp = (sh.G + 3) / 4;
+  a.d = sh.d;
   a.scale = sh.scale;
   dim3 grid(sh.NB, sh.Hkv * a.n_tp, sh.B);
   kern<<<grid, fsm::kThreads, fsm::kSmemBytes, st>>>(tq, tk, tv, a);

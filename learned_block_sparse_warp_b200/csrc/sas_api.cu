@@ -9,9 +9,6 @@
 namespace sas {
 cudaError_t launch_select(const Shape& sh, const float* s, const int32_t* cache_len, int32_t* idx, float* lse,
                           int* err, cudaStream_t st);
-cudaError_t launch_fwd_mma(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* s,
-                           const int32_t* idx, const float* lse_s, uint16_t* o, float* lse_o, int* err,
-                           cudaStream_t st);
 cudaError_t launch_fwd_sm100(const Shape& sh, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                              const float* s, const int32_t* idx, const float* lse_s, uint16_t* o, float* lse_o,
                              int* err, cudaStream_t st);
@@ -163,12 +160,9 @@ sas_status sas_fwd(const sas_params* p, const sas_bf16* q, const sas_bf16* k, co
   if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(idx) || !ok_ptr(o) || !ok_opt(lse_o))
     return SAS_ERR_INVALID_ARG;
   if (!gate_inputs_ok(sh, s, lse_s)) return SAS_ERR_INVALID_ARG;
-  // d = 128: TMA + tcgen05 kernel; d = 64: warp-level tensor-core kernel
-  if (sh.d == 128)
-    return from_cuda(sas::launch_fwd_sm100(sh, q, k, v, sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, o,
-                                           lse_o, device_error_word(), static_cast<cudaStream_t>(stream)));
-  return from_cuda(sas::launch_fwd_mma(sh, q, k, v, sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, o, lse_o,
-                                       device_error_word(), static_cast<cudaStream_t>(stream)));
+  // tcgen05 kernel for d = 64 and 128 (at 64 the tensor maps zero-fill the second half of each row box)
+  return from_cuda(sas::launch_fwd_sm100(sh, q, k, v, sh.gated ? s : nullptr, idx, sh.gated ? lse_s : nullptr, o,
+                                         lse_o, device_error_word(), static_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_bwd_workspace_size(const sas_params* p, size_t* bytes) {

@@ -227,10 +227,12 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 }  // namespace sm100
 
-// Row-major bf16 matrix [rows, cols] read in 64 x 64 boxes with the 128-byte swizzle (host).
+// Row-major bf16 matrix [rows, cols] read in 64 x 64 boxes with the 128-byte swizzle (host). A box
+// that starts past cols (the second d-half of a cols = 64 matrix) reads as zeros.
 bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols);
-// bf16 [heads, N, 128] in boxes of 2 heads x 64 tokens x 64 d (host).
-bool make_tmap_bf16_3d_heads(CUtensorMap* m, const void* base, uint64_t heads, uint64_t N);
+// bf16 [heads, N, d] in boxes of 2 heads x 64 tokens x 64 d (host); at d = 64 the second
+// 64-column box of a row is past the extent and reads as zeros.
+bool make_tmap_bf16_3d_heads(CUtensorMap* m, const void* base, uint64_t heads, uint64_t N, uint64_t d);
 // fp32 [rows, N] in boxes of 2 rows x 64 values (host).
 bool make_tmap_f32_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t N);
 // bf16 [tiles, 128, 64]: one box is one whole 16 KB tile of 128 rows x 64 values (128-byte swizzle).

@@ -119,9 +119,13 @@ def test_workspace_size_and_check():
         assert fn(ctypes.byref(c), None) == INVALID
 
 
-def test_workspace_d64_has_one_form():
-    p = _p(head_dim=64)
-    assert sas.sas_bwd_workspace_size(p) == sas.sas_bwd_workspace_size_min(p)
+def test_workspace_d64_has_both_forms():
+    # the same tcgen05 passes serve d = 64: the full workspace adds the same dZ tiles (128 x 64 bf16
+    # per query block, attended block and head pair, independent of d)
+    p, p128 = _p(head_dim=64), _p(head_dim=128)
+    extra64 = sas.sas_bwd_workspace_size(p) - sas.sas_bwd_workspace_size_min(p)
+    extra128 = sas.sas_bwd_workspace_size(p128) - sas.sas_bwd_workspace_size_min(p128)
+    assert extra64 == extra128 > 0
 
 
 def test_decode_split_count_checked():
