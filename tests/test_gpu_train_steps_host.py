@@ -1,9 +1,10 @@
 """GPU: training steps end to end from host memory (sas_train_steps_host).
 
 Each step's inputs go up, the step runs, its outputs come down, with the copies
-of neighbouring steps overlapping the kernels on two device slots. With d = 128
-every kernel on the path is deterministic (the backward has no atomics), so each
-step's host outputs must equal those of the same step run on device buffers.
+of neighbouring steps overlapping the kernels on two device slots. Every kernel
+on the path is deterministic (the backward has no atomics), so each step's host
+outputs must equal those of the same step run on device buffers; they are also
+compared with the fp64 oracle directly.
 """
 import numpy as np
 import pytest
@@ -82,3 +83,34 @@ def test_host_steps_without_gate_and_shared_buffers():
     assert sas.sas_get_device_error() == 0
     for k in ("o", "lse_o", "dq", "dk", "dv"):
         assert torch.equal(ho[k], ref[k]), k
+
+
+@pytest.mark.parametrize("shape", ["tiny", "gqa4_d128"])
+def test_host_steps_match_the_oracle(shape):
+    """Each step's host outputs against the fp64 oracle directly, at the parity tolerances: the
+    tiny configuration (2 heads, d = 64, N = 1024, K = 4) and a GQA-4 d = 128 shape."""
+    import learned_block_sparse_warp_b200 as sas
+    import oracle.sas_oracle as O
+    from tests.parity_util import TOL_L, TOL_O, TOL_REL, max_abs, rel_fro
+    if shape == "tiny":
+        w = W.WORKLOADS["tiny"]
+    else:
+        w = W.custom("host_oracle", batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, seq_len=1024, top_k=4, seed=77)
+    p = sas.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
+                   seq_len=w.seq_len, top_k=w.top_k, gate_mode=sas.SAS_GATE_LOG_SOFTMAX)
+    x = W.prefill_inputs(w, with_do=True)
+    h = {k: torch.from_numpy(np.ascontiguousarray(x[k])).to(torch.bfloat16 if k != "s" else torch.float32)
+         .pin_memory() for k in ("q", "k", "v", "s", "do")}
+    ho = _host_outputs(p, True)
+    sas.sas_train_steps_host(p, [{**h, **ho}], [sas.empty_device_slot(p), sas.empty_device_slot(p)])
+    torch.cuda.synchronize()
+    assert sas.sas_get_device_error() == 0
+    f64 = {k: h[k].float().numpy().astype(np.float64) for k in ("q", "k", "v", "s", "do")}
+    idx, _ = O.prefill_select(f64["s"], w.top_k)
+    o, L = O.forward(f64["q"], f64["k"], f64["v"], f64["s"], idx)
+    dq, dk, dv, ds, _ = O.backward(f64["q"], f64["k"], f64["v"], f64["s"], idx, f64["do"])
+    got = {k: ho[k].float().numpy().astype(np.float64) for k in OUTS}
+    assert max_abs(got["o"], o) < TOL_O
+    assert max_abs(got["lse_o"], L) < TOL_L
+    for k, ref in (("dq", dq), ("dk", dk), ("dv", dv), ("ds", ds)):
+        assert rel_fro(got[k], ref) < TOL_REL, (k, rel_fro(got[k], ref))
