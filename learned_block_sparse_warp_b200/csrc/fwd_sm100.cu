@@ -14,9 +14,11 @@
 //                the Q rows once, then each selected K/V block into a
 //                4-stage shared-memory ring. Blocks are gathered by index
 //                with no copy in HBM.
-//   warps 1, 3   one MMA-issuing thread per tile (warp 1 also allocates the
+//   warps 1, 3   one MMA-issuing warp per tile (warp 1 also allocates the
 //                512 TMEM columns): S_r(b) = Q_r K_bᵀ (SS, fp32 in TMEM), then
-//                O_r += P_r(b) V_b (TS: P read from TMEM).
+//                O_r += P_r(b) V_b (TS: P read from TMEM). The whole warp
+//                walks the loop and waits; elect.sync picks the lane that
+//                issues, so the operands stay warp-uniform.
 //   warps 4-7    softmax of tile 0; warps 8-11 softmax of tile 1. Each thread
 //                owns one row: it reads the block's 64 logits from TMEM,
 //                masks the current block causally, adds the block's log-gate,
@@ -24,6 +26,10 @@
 //                consumed S columns. O is rescaled in TMEM only when the row
 //                max grows by more than 2^8, so the result is exact and
 //                rescales are rare.
+//                With two tiles, their exponential sections take turns
+//                (tile 0 on block b, then tile 1 on block b, then tile 0 on
+//                b + 1), handed over by an mbarrier, so the two groups do
+//                not contend for the same issue slots at the same moment.
 // Each tile has two 64-column S buffers: S of block b + 1 is computed while
 // the softmax works on block b and PV of block b − 1 runs, so no tile waits
 // for its own PV before its next S.
@@ -36,7 +42,7 @@
 namespace sas {
 
 namespace fsm {
-constexpr int kThreads = 384;            // 0 TMA, 1 and 3 MMA (one per tile), 4-11 softmax
+constexpr int kThreads = 384;            // 0 TMA, 1 and 3 MMA (one warp per tile), 4-11 softmax
 constexpr int kStages = 4;               // one gathered K/V block per stage
 constexpr int kHalf = 128 * 128;         // one d-half of a 128-row Q tile: 128 rows x 128 B
 constexpr int kQBytes = 4 * kHalf;       // 2 tiles x 2 d-halves
@@ -80,7 +86,7 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
   __shared__ float lam_s[kMaxTopK + 1];
   __shared__ int nlist_s;
   __shared__ __align__(8) uint64_t bar_q, bar_full[fsm::kStages], bar_empty[fsm::kStages], bar_s[2][2], bar_p[2][2],
-      bar_pv[2][2], bar_fin;
+      bar_pv[2][2], bar_fin, bar_turn[2];
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
 
@@ -117,6 +123,8 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
           mbar_init(smem_u32(&bar_pv[r][c]), 1);
         }
       mbar_init(smem_u32(&bar_fin), n_tiles);
+      mbar_init(smem_u32(&bar_turn[0]), 4);
+      mbar_init(smem_u32(&bar_turn[1]), 4);
       fence_barrier_init();
     }
   }
@@ -162,8 +170,9 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
       }
     }
   } else if ((warp == 1 || warp == 3) && (warp >> 1) < n_tiles) {
-    // ------------------------------------------------------------ MMA issuers, one thread per tile
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuers, one warp per tile
+    // The whole warp walks the loop and waits; one elected lane issues each MMA.
+    {
       const int r = warp >> 1;
       const uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);   // q rows x kv, K = d
       const uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);  // q rows x d, K = kv; V MN-major
@@ -176,35 +185,36 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         const uint32_t so = (i % fsm::kStages) * fsm::kStageBytes;
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mma_ss(tT + (i & 1) * 64, desc_advance(dQ0, (k >> 2) * fsm::kHalf + (k & 3) * 32),
-                 desc_advance(dK0, so + (k >> 2) * fsm::kHalfKV + (k & 3) * 32), idS, k > 0 ? 1u : 0u);
-        mma_commit(smem_u32(&bar_s[r][i & 1]));
+          mma_ss_e(tT + (i & 1) * 64, desc_advance(dQ0, (k >> 2) * fsm::kHalf + (k & 3) * 32),
+                   desc_advance(dK0, so + (k >> 2) * fsm::kHalfKV + (k & 3) * 32), idS, k > 0 ? 1u : 0u);
+        mma_commit_e(smem_u32(&bar_s[r][i & 1]));
       };
       bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, a.err);
       ok = ok && mbar_wait(smem_u32(&bar_full[0]), 0, abort_flag, a.err);
+      ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok) issue_s(0);
       for (int i = 0; ok && i < nl; ++i) {
         if (i + 1 < nl) {
           const int n = i + 1;
-          if (!(ok = mbar_wait(smem_u32(&bar_full[n % fsm::kStages]), (n / fsm::kStages) & 1, abort_flag, a.err)))
-            break;
+          ok = mbar_wait(smem_u32(&bar_full[n % fsm::kStages]), (n / fsm::kStages) & 1, abort_flag, a.err);
           // PV of block n − 2 read its P from the buffer that S(n) overwrites
-          if (n >= 2 && !(ok = mbar_wait(smem_u32(&bar_pv[r][n & 1]), ((n - 2) >> 1) & 1, abort_flag, a.err)))
-            break;
+          if (ok && n >= 2) ok = mbar_wait(smem_u32(&bar_pv[r][n & 1]), ((n - 2) >> 1) & 1, abort_flag, a.err);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
           tc_fence_after();
           issue_s(n);
         }
-        if (!(ok = mbar_wait(smem_u32(&bar_p[r][i & 1]), (i >> 1) & 1, abort_flag, a.err))) break;
+        ok = mbar_wait(smem_u32(&bar_p[r][i & 1]), (i >> 1) & 1, abort_flag, a.err);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
         tc_fence_after();
         const uint32_t sv = (i % fsm::kStages) * fsm::kStageBytes;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj)  // P(i) packed over the first 32 columns of its S buffer
-          mma_ts(tO, tT + (i & 1) * 64 + jj * 8, desc_advance(dV0, sv + jj * 2048), idPV, (i > 0 || jj > 0) ? 1u : 0u);
-        mma_commit(smem_u32(&bar_pv[r][i & 1]));
-        mma_commit(smem_u32(&bar_empty[i % fsm::kStages]));
+          mma_ts_e(tO, tT + (i & 1) * 64 + jj * 8, desc_advance(dV0, sv + jj * 2048), idPV, (i > 0 || jj > 0) ? 1u : 0u);
+        mma_commit_e(smem_u32(&bar_pv[r][i & 1]));
+        mma_commit_e(smem_u32(&bar_empty[i % fsm::kStages]));
       }
-      mma_commit(smem_u32(&bar_fin));
+      mma_commit_e(smem_u32(&bar_fin));
     }
   } else if (warp >= 4 && (warp - 4) / 4 < n_tiles) {
     // ------------------------------------------------------------ softmax, one row per thread
@@ -255,6 +265,13 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
         l *= alpha;
         m_used = mx;
       }
+      if (n_tiles == 2 && (r == 1 || i > 0)) {
+        const bool got = mbar_wait(smem_u32(&bar_turn[r]), (r == 0 ? i - 1 : i) & 1, abort_flag, a.err);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+      }
       // probabilities, row sum, bf16 P over the S columns just read
       {
         const float off = lam - m_used;  // p = 2^(S·sc2 + λ − m)
@@ -276,6 +293,10 @@ __global__ void __launch_bounds__(fsm::kThreads, 1)
           }
         }
         l += s0 + s1;
+        if (n_tiles == 2) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bar_turn[r ^ 1]));
+        }
         tmem_st32(tS, pk);
       }
       if (i > 0 && __any_sync(0xffffffffu, grow)) {
