@@ -261,6 +261,40 @@ SAS_API sas_status sas_decode_paged(const sas_params* p, const sas_bf16* q, cons
 SAS_API sas_status sas_decode_combine(const sas_params* p, int n_split, const float* o_part, const float* lse_part,
                               sas_bf16* o, float* lse_o, void* stream);
 
+/* The whole decode step in one launch: the Top-K select of sas_topk_select
+ * (decode form) on s, the attention of sas_decode over the current block and
+ * the picks, and the merge of sas_decode_combine. SAS explainer §仕組み,
+ * Algorithm 2: scores pick the Top-K history blocks, attention runs over them
+ * and the current block; the gate modes apply as in sas_decode.
+ *
+ * One cluster of up to 8 CTAs serves each (sequence, KV head) row. Each CTA
+ * selects the row's blocks itself, attends to its share of the ordered list
+ * and keeps its partial in shared memory; the cluster merges the partials over
+ * distributed shared memory. No partial goes to HBM and no workspace is taken.
+ *
+ *   q, kc, vc, cache_len  as in sas_decode.
+ *   s      fp32 [B, Hkv, NKB], always read (it drives the selection).
+ *   idx    int32 [B, Hkv, K]. Output, may be NULL: the picks, ascending, −1
+ *          padded, bit for bit those of sas_topk_select.
+ *   lse_s  fp32 [B, Hkv]. Output, may be NULL: LSE of the history scores.
+ *   o      bf16 [B, Hq, d]. Output.
+ *   lse_o  fp32 [B, Hq]. Output, may be NULL.
+ * Limits: G <= 8, K <= 255 and NKB <= 2048 (the row's keys and picks live in
+ * shared memory); other shapes return SAS_ERR_UNSUPPORTED before any launch
+ * and are served by the separate calls. A cache_len outside [1, seq_len]
+ * raises SAS_ERR_DEVICE_INDEX and is clamped. */
+SAS_API sas_status sas_decode_fused(const sas_params* p, const sas_bf16* q, const sas_bf16* kc, const sas_bf16* vc,
+                                    const int32_t* cache_len, const float* s, int32_t* idx, float* lse_s, sas_bf16* o,
+                                    float* lse_o, void* stream);
+
+/* sas_decode_fused over the paged cache of sas_decode_paged (k_pages, v_pages,
+ * n_pages, block_table as there). Only the table entries of the blocks the
+ * step reads are read. */
+SAS_API sas_status sas_decode_fused_paged(const sas_params* p, const sas_bf16* q, const sas_bf16* k_pages,
+                                          const sas_bf16* v_pages, int n_pages, const int32_t* block_table,
+                                          const int32_t* cache_len, const float* s, int32_t* idx, float* lse_s,
+                                          sas_bf16* o, float* lse_o, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Selector scoring fused with Top-K for long decode caches (SAS summary
  * §전제와 한계: in decode, the selector's scoring and the Top-K ranking grow

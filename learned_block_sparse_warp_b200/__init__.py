@@ -28,7 +28,8 @@ __all__ = [
     "sas_decode_combine", "sas_decode_paged", "sas_decode_noalloc", "sas_get_device_error", "sas_status_string",
     "sas_version",
     "DecodeGraph", "sas_selftest_wait_timeout", "sas_block_mean_keys", "sas_decode_select_scored",
-    "decode_step_scored", "sas_train_steps_host", "empty_device_slot",
+    "decode_step_scored", "sas_train_steps_host", "empty_device_slot", "sas_decode_fused", "sas_decode_fused_paged",
+    "decode_step_fused",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
@@ -86,6 +87,8 @@ def _load() -> ctypes.CDLL:
         "sas_decode_combine": [P, ctypes.c_int, vp, vp, vp, vp, vp],
         "sas_get_device_error": [vp, ctypes.POINTER(ctypes.c_int)],
         "sas_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp],
+        "sas_decode_fused": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "sas_decode_fused_paged": [P, vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp],
         "sas_selftest_wait_timeout": [vp],
         "sas_block_mean_keys": [P, vp, vp, vp, vp],
         "sas_decode_select_scored": [P, vp, vp, vp, vp, vp, vp, vp],
@@ -268,6 +271,31 @@ def sas_decode_noalloc(p: Params, q, kc, vc, cache_len, s, o, lse_o=None, stream
         _stream(stream)))
 
 
+def sas_decode_fused(p: Params, q, kc, vc, cache_len, s, o, idx=None, lse_s=None, lse_o=None, stream=None) -> None:
+    """Whole decode step in one launch: select, attention, merge (idx, lse_s and lse_o are optional outputs)."""
+    B, Hq, Hkv, d = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim
+    sh = _shapes(p, True)
+    _check("sas_decode_fused", lib.sas_decode_fused(
+        ctypes.byref(p.c()), _ptr(q, bf16, (B, Hq, d), "q"), _ptr(kc, bf16, (B, Hkv, p.seq_len, d), "kc"),
+        _ptr(vc, bf16, (B, Hkv, p.seq_len, d), "vc"), _ptr(cache_len, i32, (B,), "cache_len"),
+        _ptr(s, f32, sh["s"], "s"), _ptr(idx, i32, sh["idx"], "idx"), _ptr(lse_s, f32, sh["lse_s"], "lse_s"),
+        _ptr(o, bf16, (B, Hq, d), "o"), _ptr(lse_o, f32, (B, Hq), "lse_o"), _stream(stream)))
+
+
+def sas_decode_fused_paged(p: Params, q, k_pages, v_pages, block_table, cache_len, s, o, idx=None, lse_s=None,
+                           lse_o=None, stream=None) -> None:
+    """sas_decode_fused over a paged cache: k_pages/v_pages [n_pages, Hkv, 64, d], block_table int32 [B, NKB]."""
+    B, Hq, Hkv, d = p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim
+    n_pages = int(k_pages.shape[0]) if k_pages is not None else 0
+    sh = _shapes(p, True)
+    _check("sas_decode_fused_paged", lib.sas_decode_fused_paged(
+        ctypes.byref(p.c()), _ptr(q, bf16, (B, Hq, d), "q"), _ptr(k_pages, bf16, (n_pages, Hkv, p.block, d), "k_pages"),
+        _ptr(v_pages, bf16, (n_pages, Hkv, p.block, d), "v_pages"), n_pages,
+        _ptr(block_table, i32, (B, p.n_blocks), "block_table"), _ptr(cache_len, i32, (B,), "cache_len"),
+        _ptr(s, f32, sh["s"], "s"), _ptr(idx, i32, sh["idx"], "idx"), _ptr(lse_s, f32, sh["lse_s"], "lse_s"),
+        _ptr(o, bf16, (B, Hq, d), "o"), _ptr(lse_o, f32, (B, Hq), "lse_o"), _stream(stream)))
+
+
 def sas_block_mean_keys(p: Params, k, kmean, cache_len=None, stream=None) -> None:
     """k̄[b, h, m] = mean of block m's 64 keys (bf16). With cache_len, only each sequence's just-completed block."""
     B, Hkv, d = p.batch, p.n_kv_heads, p.head_dim
@@ -411,6 +439,13 @@ def decode_step(p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, str
     sas_decode_combine(p, n_split, out["o_part"], out["lse_part"], out["o"], out["lse_o"], stream=stream)
 
 
+def decode_step_fused(p: Params, q, kc, vc, cache_len, s, out: dict, stream=None) -> None:
+    """One decode step in one launch (select, attention, merge); fills out["o"], out["lse_o"], out["idx"] and
+    out["lse_s"] when present."""
+    sas_decode_fused(p, q, kc, vc, cache_len, s, out["o"], idx=out.get("idx"), lse_s=out.get("lse_s"),
+                     lse_o=out.get("lse_o"), stream=stream)
+
+
 def decode_step_scored(p: Params, q, kc, vc, kmean, cache_len, s, n_split: int, out: dict, stream=None) -> None:
     """A decode step that scores its own history: update the block means of any block the newest token
     completed, score and select in one launch (s is written), split-K attention, merge."""
@@ -428,12 +463,17 @@ class DecodeGraph:
     next step's query, scores and cache lengths into the same tensors and
     calls ``replay()``. One replay is three kernel launches with no host work
     between them. The three kernels are chained by programmatic dependent
-    launch, so each one's launch overlaps the tail of the one before.
+    launch, so each one's launch overlaps the tail of the one before. With
+    ``fused=True`` a replay is the single launch of sas_decode_fused.
     """
 
-    def __init__(self, p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, stream=None, kmean=None):
-        # with kmean, the step scores its own history (decode_step_scored) and s is an output
-        if kmean is None:
+    def __init__(self, p: Params, q, kc, vc, cache_len, s, n_split: int, out: dict, stream=None, kmean=None,
+                 fused: bool = False):
+        # with kmean, the step scores its own history (decode_step_scored) and s is an output; with fused, the
+        # step is the single launch of sas_decode_fused (n_split is then unused)
+        if fused and kmean is None:
+            self.step, self.args = decode_step_fused, (p, q, kc, vc, cache_len, s, out)
+        elif kmean is None:
             self.step, self.args = decode_step, (p, q, kc, vc, cache_len, s, n_split, out)
         else:
             self.step, self.args = decode_step_scored, (p, q, kc, vc, kmean, cache_len, s, n_split, out)

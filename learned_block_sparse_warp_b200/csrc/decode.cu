@@ -27,15 +27,22 @@
 // scores 16 of the block's 64 tokens. Row maxima and sums are exchanged
 // through shared memory. P goes through a swizzled 16 x 64 bf16 tile, and
 // each warp then accumulates PV for a quarter of the head dimension.
+#include <cooperative_groups.h>
+
 #include <type_traits>
 
 #include "common.cuh"
 
 namespace sas {
 
+namespace cg = cooperative_groups;
+
 namespace dec {
 constexpr int kThreads = 128;
 constexpr int kMaxTasks = kMaxDecodeBlocksPerSplit;  // task slots per chunk of items (2 CTAs per SM at d = 128)
+constexpr int kFusedMaxK = 255;     // the fused step keeps the whole selected list in shared memory
+constexpr int kFusedMaxNB = 2048;   // and the row's keys (4 bytes each) in one ring stage
+constexpr int kMaxCluster = 8;      // portable cluster size
 }  // namespace dec
 
 struct DecodeArgs {
@@ -54,6 +61,128 @@ struct DecodeArgs {
   int B, Hkv, Lmax, K, gate, gated, outside, n_split, per_max, items_per_chunk;
   float scale;
 };
+
+struct DecodeFusedArgs {
+  const uint16_t* q;
+  const uint16_t* kc;
+  const uint16_t* vc;
+  const int32_t* cache_len;
+  const float* s;
+  const int32_t* table;  // paged cache block table, or null for the dense cache
+  int n_pages;
+  int32_t* idx;    // [B, Hkv, K] picks, may be null
+  float* lse_s;    // [B, Hkv], may be null
+  uint16_t* o;     // [B, Hq, d]
+  float* lse_o;    // [B, Hq], may be null
+  int* err;
+  int B, Hkv, Lmax, K, gate, gated, outside, need_lse;
+  float scale;
+};
+
+// The running state of one item's online softmax in one thread: the O fragments
+// of this warp's d columns (rows are heads; rows >= G are padding), the row max
+// and sum of head g_row (log2 domain, the same in every warp), and the A
+// fragments of the padded query rows.
+template <int D>
+struct DecAcc {
+  float o[D / 32][4];
+  float m, l;
+  uint32_t qa[D / 16][4];
+};
+
+// One 64-token block of an item, run by all 128 threads: S = q Kᵀ on mma.sync
+// (each warp scores 16 tokens), the block's softmax update with the maxima and
+// sums exchanged through shared memory, P through the swizzled tile at sP, and
+// O += P V over each warp's quarter of d. `st` is the ring stage that holds the
+// block's K and V tiles (and, for the item's first block, its query rows).
+// Tokens past ntok are masked. lam2 biases the logits (log2 domain); gw
+// weights P·V. Contains two __syncthreads.
+template <int D, int G>
+__device__ __forceinline__ void dec_block(DecAcc<D>& A, uint32_t st, uint32_t sP, int ntok, float lam2, float gw,
+                                          bool first, float sc2, float (*red_max)[8], float (*red_sum)[8]) {
+  constexpr int CH = D / 8;             // 16-byte chunks per row
+  constexpr int TILEB = kBlock * D * 2;  // one 64-token tile
+  constexpr int DW = D / 4;             // d columns per warp in PV
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g_row = lane >> 2;  // the head this thread's C-fragment row 0 belongs to
+  if (first) {
+#pragma unroll
+    for (int j = 0; j < DW / 8; ++j) A.o[j][0] = A.o[j][1] = A.o[j][2] = A.o[j][3] = 0.f;
+    A.m = -INFINITY;
+    A.l = 0.f;
+    // this stage holds the item's query rows; keep their A fragments in registers
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      ldsm_x4(st + 2 * TILEB + swz<CH>(lane & 15, 2 * kk + (lane >> 4)), A.qa[kk][0], A.qa[kk][1], A.qa[kk][2], A.qa[kk][3]);
+  }
+  // S = q Kᵀ for this warp's 16 tokens (two n8 tiles); rows are heads
+  float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4(st + swz<CH>(16 * warp + (lane & 7) + ((lane >> 4) << 3), 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
+    mma_bf16_16816(sacc[0], A.qa[kk], b0, b1);
+    mma_bf16_16816(sacc[1], A.qa[kk], b2, b3);
+  }
+  // gated logits (log2 domain) of head g_row; tokens past ntok are masked
+  float z[4];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int n = 0; n < 2; ++n)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int tok = 16 * warp + 8 * n + 2 * (lane & 3) + e;
+      const float v = tok < ntok ? fmaf(sacc[n][e], sc2, lam2) : -INFINITY;
+      z[2 * n + e] = v;
+      mx = fmaxf(mx, v);
+    }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  if ((lane & 3) == 0 && g_row < 8) red_max[warp][g_row] = mx;
+  __syncthreads();
+  const float m_blk = fmaxf(fmaxf(red_max[0][g_row], red_max[1][g_row]), fmaxf(red_max[2][g_row], red_max[3][g_row]));
+  const float m_new = fmaxf(A.m, m_blk);
+  const float alpha = (A.m == -INFINITY) ? 0.f : exp2f(A.m - m_new);
+  float ps = 0.f;
+  float pv[4];
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    pv[x] = (z[x] == -INFINITY) ? 0.f : exp2f(z[x] - m_new);
+    ps += pv[x];
+  }
+  ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+  ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+  if ((lane & 3) == 0 && g_row < 8) red_sum[warp][g_row] = ps;
+  // P (bf16) of head g_row at tokens 16 warp + 8 n + 2 (lane & 3) + {0, 1}
+#pragma unroll
+  for (int n = 0; n < 2; ++n) {
+    const int tok = 16 * warp + 8 * n + 2 * (lane & 3);
+    const uint32_t addr = sP + swz<8>(g_row, tok >> 3) + (tok & 7) * 2;
+    asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(addr), "r"(pack_bf16x2(pv[2 * n] * gw, pv[2 * n + 1] * gw)));
+  }
+#pragma unroll
+  for (int j = 0; j < DW / 8; ++j) {
+    A.o[j][0] *= alpha;
+    A.o[j][1] *= alpha;
+  }
+  __syncthreads();
+  A.l = A.l * alpha + ((red_sum[0][g_row] + red_sum[1][g_row]) + (red_sum[2][g_row] + red_sum[3][g_row]));
+  A.m = m_new;
+  // O += P V over this warp's d columns [DW warp, DW warp + DW)
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    uint32_t pa[4];
+    ldsm_x4(sP + swz<8>(lane & 15, 2 * kk + (lane >> 4)), pa[0], pa[1], pa[2], pa[3]);
+#pragma unroll
+    for (int dp = 0; dp < DW / 16; ++dp) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(st + TILEB + swz<CH>(16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3), (DW / 8) * warp + 2 * dp + (lane >> 4)),
+                b0, b1, b2, b3);
+      mma_bf16_16816(A.o[2 * dp], pa, b0, b1);
+      mma_bf16_16816(A.o[2 * dp + 1], pa, b2, b3);
+    }
+  }
+}
 
 template <int D, int G, int STAGES>
 __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs a) {
@@ -97,8 +226,6 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
   const int my_items = (n_items > int(blockIdx.x)) ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
   const int g_row = lane >> 2;  // the head this thread's C-fragment row 0 belongs to
 
-  float oacc[DW / 8][4];
-  float m_run = -INFINITY, l_run = 0.f;  // for head g_row (log2 domain), same in every warp
 
   for (int chunk0 = 0; chunk0 < my_items; chunk0 += a.items_per_chunk) {
     const int n_chunk = min(a.items_per_chunk, my_items - chunk0);
@@ -212,108 +339,31 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
       if (s < nt) issue(s);
       cp_async_commit();
     }
-    uint32_t qa[D / 16][4];  // A fragments of the padded query rows (rows >= G are zero)
+    DecAcc<D> acc;  // the running O fragments, max and sum of the item in flight
     for (int task = 0; task < nt; ++task) {
       if (task + STAGES - 1 < nt) issue(task + STAGES - 1);
       cp_async_commit();
       cp_async_wait<STAGES - 1>();
       __syncthreads();
       const uint32_t st = ring + (task % STAGES) * STAGEB;
-      const int ntok = t_ntok[task];
       // the gate inside the softmax biases the logits by log2 g; outside, it weights P·V by g
       const float lam2 = a.outside ? 0.f : t_lam[task];
       const float gw = a.outside ? exp2f(t_lam[task]) : 1.f;
       const int flags = t_flags[task];
-      if (flags & 1) {
-#pragma unroll
-        for (int j = 0; j < DW / 8; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
-        m_run = -INFINITY;
-        l_run = 0.f;
-        // this stage holds the item's query rows; keep their A fragments in registers
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          ldsm_x4(st + 2 * TILEB + swz<CH>(lane & 15, 2 * kk + (lane >> 4)), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-      }
-      // S = q Kᵀ for this warp's 16 tokens (two n8 tiles); rows are heads
-      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(st + swz<CH>(16 * warp + (lane & 7) + ((lane >> 4) << 3), 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
-        mma_bf16_16816(sacc[0], qa[kk], b0, b1);
-        mma_bf16_16816(sacc[1], qa[kk], b2, b3);
-      }
-      // gated logits (log2 domain) of head g_row; tokens past ntok are masked
-      float z[4];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int n = 0; n < 2; ++n)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tok = 16 * warp + 8 * n + 2 * (lane & 3) + e;
-          const float v = tok < ntok ? fmaf(sacc[n][e], sc2, lam2) : -INFINITY;
-          z[2 * n + e] = v;
-          mx = fmaxf(mx, v);
-        }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      if ((lane & 3) == 0 && g_row < 8) red_max[warp][g_row] = mx;
-      __syncthreads();
-      const float m_blk = fmaxf(fmaxf(red_max[0][g_row], red_max[1][g_row]), fmaxf(red_max[2][g_row], red_max[3][g_row]));
-      const float m_new = fmaxf(m_run, m_blk);
-      const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_new);
-      float ps = 0.f;
-      float pv[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        pv[x] = (z[x] == -INFINITY) ? 0.f : exp2f(z[x] - m_new);
-        ps += pv[x];
-      }
-      ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-      ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-      if ((lane & 3) == 0 && g_row < 8) red_sum[warp][g_row] = ps;
-      // P (bf16) of head g_row at tokens 16 warp + 8 n + 2 (lane & 3) + {0, 1}
-#pragma unroll
-      for (int n = 0; n < 2; ++n) {
-        const int tok = 16 * warp + 8 * n + 2 * (lane & 3);
-        const uint32_t addr = sP + swz<8>(g_row, tok >> 3) + (tok & 7) * 2;
-        asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(addr), "r"(pack_bf16x2(pv[2 * n] * gw, pv[2 * n + 1] * gw)));
-      }
-#pragma unroll
-      for (int j = 0; j < DW / 8; ++j) {
-        oacc[j][0] *= alpha;
-        oacc[j][1] *= alpha;
-      }
-      __syncthreads();
-      l_run = l_run * alpha + ((red_sum[0][g_row] + red_sum[1][g_row]) + (red_sum[2][g_row] + red_sum[3][g_row]));
-      m_run = m_new;
-      // O += P V over this warp's d columns [DW warp, DW warp + DW)
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t pa[4];
-        ldsm_x4(sP + swz<8>(lane & 15, 2 * kk + (lane >> 4)), pa[0], pa[1], pa[2], pa[3]);
-#pragma unroll
-        for (int dp = 0; dp < DW / 16; ++dp) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(st + TILEB + swz<CH>(16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3), (DW / 8) * warp + 2 * dp + (lane >> 4)),
-                    b0, b1, b2, b3);
-          mma_bf16_16816(oacc[2 * dp], pa, b0, b1);
-          mma_bf16_16816(oacc[2 * dp + 1], pa, b2, b3);
-        }
-      }
+      dec_block<D, G>(acc, st, sP, t_ntok[task], lam2, gw, (flags & 1) != 0, sc2, red_max, red_sum);
       if (flags & 2) {  // the item's last block: write its normalised partial for the G heads
         const int it = t_item[task];
         const int split = it % a.n_split, bh = it / a.n_split;
         if (g_row < G) {
           const size_t row = (size_t(bh) * G + g_row) * a.n_split + split;
-          const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+          const float inv = acc.l > 0.f ? 1.f / acc.l : 0.f;
 #pragma unroll
           for (int j = 0; j < DW / 8; ++j) {
             const int col = DW * warp + 8 * j + 2 * (lane & 3);
-            *reinterpret_cast<float2*>(a.o_part + row * D + col) = make_float2(oacc[j][0] * inv, oacc[j][1] * inv);
+            *reinterpret_cast<float2*>(a.o_part + row * D + col) = make_float2(acc.o[j][0] * inv, acc.o[j][1] * inv);
           }
           if (warp == 0 && (lane & 3) == 0)
-            a.lse_part[row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+            a.lse_part[row] = acc.l > 0.f ? (acc.m + log2f(acc.l)) * kLn2 : -INFINITY;
         }
       }
       __syncthreads();
@@ -321,6 +371,332 @@ __global__ void __launch_bounds__(dec::kThreads) decode_split_kernel(DecodeArgs 
     cp_async_wait<0>();
     __syncthreads();
   }
+}
+
+// ---------------------------------------------------------------------------
+// The whole decode step in one launch (sas_decode_fused): one cluster of CS
+// CTAs per (sequence, KV head) row. Every CTA of the cluster selects the row's
+// Top-K blocks itself (the row is 2 KB at 32K, so the redundant work is cheaper
+// than a hand-over) while the first CTA's load of the current block is in
+// flight. Each CTA then streams its share of the ordered list [current block,
+// picks...] through the same cp.async ring and block step as the split kernel,
+// and leaves its unnormalised partial (O fragments, row max, row sum) in its own
+// shared memory. After a cluster barrier every CTA merges a slice of the G x d
+// outputs from all partials over distributed shared memory, so no partial
+// touches HBM and no second kernel runs.
+
+// Exclusive sum over the 128 threads of the CTA (tot gets the total). Contains
+// two __syncthreads; wtot holds 4 ints of shared memory.
+__device__ __forceinline__ int cta_excl_sum(int v, int* wtot, int& tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += u;
+  }
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  int before = incl - v;
+  tot = 0;
+#pragma unroll
+  for (int w = 0; w < dec::kThreads / 32; ++w) {
+    before += (w < warp) ? wtot[w] : 0;
+    tot += wtot[w];
+  }
+  __syncthreads();
+  return before;
+}
+
+// The n-th largest of key[0, c) in shared memory (0 < n < c), by four 8-bit
+// radix passes from the most significant byte: each pass histograms the keys
+// that match the digits fixed so far and fixes the digit at which the count
+// from the top reaches the number still needed. Returns the threshold key;
+// need_eq gets how many keys equal to it belong to the n largest, and eq_cnt
+// how many keys equal it. (Plain shared atomics: aggregating equal digits
+// within a warp first, by match.any, measured slower on sm_100a.)
+__device__ uint32_t cta_kth_key(const uint32_t* key, int c, int n, int* hist, int* xch, int& need_eq, int& eq_cnt) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t prefix = 0u;
+  int need = n;
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += dec::kThreads) hist[i] = 0;
+    __syncthreads();
+    for (int m = tid; m < c; m += dec::kThreads) {
+      const uint32_t k = key[m];
+      if (pass == 0 || ((k ^ prefix) >> (shift + 8)) == 0u) atomicAdd(&hist[(k >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {  // lane owns bins [8 lane, 8 lane + 8); counts run from the top bin down
+      int cnt[8], own = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        cnt[u] = hist[8 * lane + u];
+        own += cnt[u];
+      }
+      int incl = own;  // own plus every lane above
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_down_sync(0xffffffffu, incl, off);
+        if (lane + off < 32) incl += u;
+      }
+      int acc = incl - own;  // keys in bins above this lane's
+      if (acc < need && need <= incl) {
+#pragma unroll
+        for (int u = 7; u >= 0; --u) {
+          if (acc + cnt[u] >= need) {
+            xch[0] = 8 * lane + u;
+            xch[1] = need - acc;
+            xch[2] = cnt[u];
+            break;
+          }
+          acc += cnt[u];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= uint32_t(xch[0]) << shift;
+    need = xch[1];
+  }
+  need_eq = need;
+  eq_cnt = xch[2];
+  return prefix;
+}
+
+template <int D, int G, int STAGES>
+__global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFusedArgs a) {
+  constexpr int CH = D / 8;
+  constexpr int ROWB = D * 2;
+  constexpr int TILEB = kBlock * ROWB;
+  constexpr int QB = 16 * ROWB;
+  constexpr int STAGEB = 2 * TILEB + QB;
+  constexpr int DW = D / 4;
+  static_assert(dec::kFusedMaxNB * 4 + 512 * 4 <= STAGEB, "keys, histogram and picks fit one ring stage");
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int sel_s[dec::kFusedMaxK];         // the row's picks, ascending
+  __shared__ float lam_s[dec::kFusedMaxK + 1];   // log2 gate of each of this CTA's tasks
+  __shared__ int xch_s[3], wtot_s[dec::kThreads / 32], napp_s;
+  __shared__ float redf_s[dec::kThreads / 32];
+  __shared__ float red_max[4][8], red_sum[4][8];
+  __shared__ __align__(128) uint16_t p_s[16 * kBlock];
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CS = int(cluster.num_blocks()), rank = int(cluster.block_rank());
+  const int bh = int(blockIdx.x) / CS;
+  const int b = bh / a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g_row = lane >> 2;
+  const int NB = a.Lmax / kBlock;
+  const float sc2 = a.scale * kLog2e;
+  const uint32_t ring = smem_u32(smem);
+  const uint32_t sP = smem_u32(p_s);
+
+  griddep_launch_dependents();
+  if (tid == 0) napp_s = 0;
+  for (int i = tid; i < STAGES * (16 - G) * CH; i += dec::kThreads) {  // padding rows, as in the split kernel
+    const int stg = i / ((16 - G) * CH), rem = i % ((16 - G) * CH);
+    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(ring + stg * STAGEB + 2 * TILEB +
+                                                                  swz<CH>(G + rem / CH, rem % CH)),
+                 "r"(0));
+  }
+  for (int i = tid; i < 16 * kBlock / 8; i += dec::kThreads)
+    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(sP + i * 16), "r"(0));
+  griddep_wait();  // q, the caches, the scores and cache_len may come from the work just before
+
+  int L = a.cache_len[b];
+  if (L < 1 || L > a.Lmax) {
+    if (tid == 0) raise_error(a.err, SAS_ERR_DEVICE_INDEX);
+    L = max(1, min(L, a.Lmax));
+  }
+  const int c = (L - 1) / kBlock;  // the current block; history blocks are [0, c)
+  const int n = min(a.K, c);
+  const float* srow = a.s + size_t(bh) * NB;
+
+  // ---- this CTA's share of the ordered list [c, picks...]
+  const int nl = 1 + n;
+  const int share = (nl + CS - 1) / CS;
+  const int p0 = min(rank * share, nl);
+  const int nt = min(p0 + share, nl) - p0;
+  auto issue = [&](int j) {
+    const uint32_t st = ring + (j % STAGES) * STAGEB;
+    const int pos = p0 + j;
+    const int m = pos == 0 ? c : sel_s[pos - 1];
+    const int ntok = pos == 0 ? L - c * kBlock : kBlock;
+    int blk = bh * NB + m;  // dense cache [B, Hkv, Lmax, d]
+    if (a.table != nullptr) {  // paged cache [n_pages, Hkv, 64, d]
+      int pg = a.table[size_t(b) * NB + m];
+      if (pg < 0 || pg >= a.n_pages) {
+        raise_error(a.err, SAS_ERR_DEVICE_INDEX);
+        pg = 0;
+      }
+      blk = pg * a.Hkv + bh % a.Hkv;
+    }
+    const size_t row0 = size_t(blk) * kBlock;
+    const uint16_t* kb = a.kc + row0 * D;
+    const uint16_t* vb = a.vc + row0 * D;
+#pragma unroll 4
+    for (int i = tid; i < kBlock * CH; i += dec::kThreads) {
+      const int r = i / CH, ch = i % CH;
+      const int nb = r < ntok ? 16 : 0;
+      const size_t off = r < ntok ? size_t(r) * D + ch * 8 : 0;
+      cp_async16_zfill(st + swz<CH>(r, ch), kb + off, nb);
+      cp_async16_zfill(st + TILEB + swz<CH>(r, ch), vb + off, nb);
+    }
+    if (j == 0) {  // the first block of the CTA brings the G query rows
+      const uint16_t* qb = a.q + size_t(bh) * G * D;
+      for (int i = tid; i < G * CH; i += dec::kThreads)
+        cp_async16(st + 2 * TILEB + swz<CH>(i / CH, i % CH), qb + (i / CH) * D + (i % CH) * 8);
+    }
+  };
+
+  // the first CTA of the cluster starts on the current block, which needs no selection
+  if (p0 == 0) {
+    if (nt > 0) issue(0);
+    cp_async_commit();
+  }
+  // ---- selection: keys of the history scores in the last ring stage (not loaded before the loop)
+  uint32_t* key_s = reinterpret_cast<uint32_t*>(smem + (STAGES - 1) * STAGEB);
+  int* hist_s = reinterpret_cast<int*>(key_s + dec::kFusedMaxNB);
+  float mx = -INFINITY;
+  for (int m = tid; m < c; m += dec::kThreads) {
+    const float v = __ldg(srow + m);
+    key_s[m] = score_key(v) + 1u;  // >= 1, so the threshold 1 takes every block
+    mx = fmaxf(mx, v);
+  }
+  float lse = 0.f;
+  if (a.need_lse) {  // LSE of the history scores, as the select kernels take it
+    mx = warp_max(mx);
+    if (lane == 0) redf_s[warp] = mx;
+    __syncthreads();
+    mx = fmaxf(fmaxf(redf_s[0], redf_s[1]), fmaxf(redf_s[2], redf_s[3]));
+    __syncthreads();
+    float sum = 0.f;
+    if (mx != -INFINITY)
+      for (int m = tid; m < c; m += dec::kThreads) sum += expf(__ldg(srow + m) - mx);
+    sum = warp_sum(sum);
+    if (lane == 0) redf_s[warp] = sum;
+    __syncthreads();
+    const float tot = (redf_s[0] + redf_s[1]) + (redf_s[2] + redf_s[3]);
+    lse = (c == 0 || mx == -INFINITY) ? -INFINITY : mx + logf(tot);
+  }
+  __syncthreads();  // every key is in place
+  const bool all = (n == c), none = (n == 0);
+  int need_eq = 0, eq_cnt = 0;
+  const uint32_t thr = (all || none) ? 1u : cta_kth_key(key_s, c, n, hist_s, xch_s, need_eq, eq_cnt);
+  if (!none && (all || need_eq == eq_cnt)) {
+    // no tie is cut at the threshold: the picks are exactly the keys >= thr. They
+    // are appended in any order, then each is placed by the number of smaller picks.
+    int* app_s = hist_s + 256;
+    for (int m = tid; m < c; m += dec::kThreads)
+      if (key_s[m] >= thr) app_s[atomicAdd(&napp_s, 1)] = m;
+    __syncthreads();
+    for (int i = tid; i < n; i += dec::kThreads) {
+      const int v = app_s[i];
+      int r = 0;
+      for (int j = 0; j < n; ++j) r += app_s[j] < v ? 1 : 0;
+      sel_s[r] = v;
+    }
+  } else if (!none) {
+    // ties cut at the threshold, taken from the lowest block index: each thread
+    // owns a contiguous run of blocks, and two block-wide scans place the picks
+    const int per = (c + dec::kThreads - 1) / dec::kThreads;
+    const int lo = min(c, tid * per), hi = min(c, lo + per);
+    int eq = 0;
+    for (int m = lo; m < hi; ++m) eq += key_s[m] == thr ? 1 : 0;
+    int tot = 0;
+    const int eq0 = cta_excl_sum(eq, wtot_s, tot);
+    int take = 0;
+    for (int m = lo, e = eq0; m < hi; ++m) {
+      const uint32_t k = key_s[m];
+      const bool is_eq = k == thr;
+      take += (k > thr || (is_eq && e < need_eq)) ? 1 : 0;
+      e += is_eq ? 1 : 0;
+    }
+    int pos = cta_excl_sum(take, wtot_s, tot);
+    for (int m = lo, e = eq0; m < hi; ++m) {
+      const uint32_t k = key_s[m];
+      const bool is_eq = k == thr;
+      if (k > thr || (is_eq && e < need_eq)) sel_s[pos++] = m;
+      e += is_eq ? 1 : 0;
+    }
+  }
+  __syncthreads();
+  if (rank == 0) {
+    if (a.idx != nullptr)
+      for (int i = tid; i < a.K; i += dec::kThreads) a.idx[size_t(bh) * a.K + i] = i < n ? sel_s[i] : -1;
+    if (a.lse_s != nullptr && tid == 0) a.lse_s[bh] = lse;
+  }
+  for (int j = tid; j < nt; j += dec::kThreads) {
+    const int pos = p0 + j;
+    lam_s[j] = (pos > 0 && a.gated) ? gate_lam2(a.gate, __ldg(srow + sel_s[pos - 1]), lse) : 0.f;
+  }
+  __syncthreads();  // lam_s is written, and the keys' stage is free for the ring
+
+  DecAcc<D> acc;
+#pragma unroll
+  for (int j = 0; j < DW / 8; ++j) acc.o[j][0] = acc.o[j][1] = acc.o[j][2] = acc.o[j][3] = 0.f;
+  acc.m = -INFINITY;
+  acc.l = 0.f;
+  if (p0 != 0) {  // the other CTAs' first block is a pick
+    if (nt > 0) issue(0);
+    cp_async_commit();
+  }
+#pragma unroll
+  for (int s = 1; s < STAGES - 1; ++s) {
+    if (s < nt) issue(s);
+    cp_async_commit();
+  }
+  for (int j = 0; j < nt; ++j) {
+    if (j + STAGES - 1 < nt) issue(j + STAGES - 1);
+    cp_async_commit();
+    cp_async_wait<STAGES - 1>();
+    __syncthreads();
+    const float lam2 = a.outside ? 0.f : lam_s[j];
+    const float gw = a.outside ? exp2f(lam_s[j]) : 1.f;
+    dec_block<D, G>(acc, ring + (j % STAGES) * STAGEB, sP, (p0 + j) == 0 ? L - c * kBlock : kBlock, lam2, gw, j == 0,
+                    sc2, red_max, red_sum);
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // ---- the partial of this CTA, unnormalised, in its first ring stage: m[G], l[G], o[G][D]
+  float* part = reinterpret_cast<float*>(smem);
+  if (g_row < G) {
+#pragma unroll
+    for (int j = 0; j < DW / 8; ++j) {
+      const int col = DW * warp + 8 * j + 2 * (lane & 3);
+      *reinterpret_cast<float2*>(part + 16 + g_row * D + col) = make_float2(acc.o[j][0], acc.o[j][1]);
+    }
+    if (warp == 0 && (lane & 3) == 0) {
+      part[g_row] = acc.m;
+      part[8 + g_row] = acc.l;
+    }
+  }
+  cluster.sync();  // every partial of the cluster is in place
+  // ---- merge: CTA `rank` writes pairs of d columns rank·128 + tid, + CS·128, ...
+  for (int e = rank * dec::kThreads + tid; e < G * D / 2; e += CS * dec::kThreads) {
+    const int g = (2 * e) / D, col = (2 * e) % D;
+    float M = -INFINITY;
+    for (int r = 0; r < CS; ++r) M = fmaxf(M, cluster.map_shared_rank(part, r)[g]);
+    float den = 0.f, n0 = 0.f, n1 = 0.f;
+    for (int r = 0; r < CS; ++r) {
+      const float* pr = cluster.map_shared_rank(part, r);
+      const float mr = pr[g];
+      const float w = (mr == -INFINITY) ? 0.f : exp2f(mr - M);
+      const float2 ov = *reinterpret_cast<const float2*>(pr + 16 + g * D + col);
+      den = fmaf(w, pr[8 + g], den);
+      n0 = fmaf(w, ov.x, n0);
+      n1 = fmaf(w, ov.y, n1);
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const size_t row = size_t(bh) * G + g;
+    *reinterpret_cast<uint32_t*>(a.o + row * D + col) = pack_bf16x2(n0 * inv, n1 * inv);
+    if (col == 0 && a.lse_o != nullptr) a.lse_o[row] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+  }
+  cluster.sync();  // no CTA leaves while another may still read its partial
 }
 
 // One warp per (sequence, query head). The lanes read the split LSEs in
@@ -464,6 +840,90 @@ cudaError_t launch_decode_paged(const Shape& sh, const uint16_t* q, const uint16
   if (sh.d == 128)
     return launch_decode_d<128>(sh, q, kp, vp, table, n_pages, cl, s, idx, lse_s, n_split, o_part, lse_part, err, st);
   return launch_decode_d<64>(sh, q, kp, vp, table, n_pages, cl, s, idx, lse_s, n_split, o_part, lse_part, err, st);
+}
+
+// The cluster size: the largest power of two of CTAs per row that keeps the
+// whole grid in one wave of resident CTAs (2 per SM at d = 128), at most 8
+// and at most one per block of the list.
+template <int D, int G>
+static cudaError_t launch_decode_fused_dg(const Shape& sh, const DecodeFusedArgs& a, cudaStream_t st) {
+  constexpr int STAGES = 3;
+  constexpr int smem = STAGES * (2 * kBlock * D * 2 + 16 * D * 2);
+  auto kern = decode_fused_kernel<D, G, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, dec::kThreads, smem)) != cudaSuccess)
+    return e;
+  const int rows = a.B * a.Hkv;
+  const int want = max(1, min(min(dec::kMaxCluster, a.K + 1), (sms * max(1, per_sm)) / rows));
+  int cs = 1;
+  while (cs * 2 <= want) cs *= 2;  // a power of two
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows * cs);
+  cfg.blockDim = dim3(dec::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if ((e = cudaLaunchKernelEx(&cfg, kern, a)) != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_decode_fused_d(const Shape& sh, const DecodeFusedArgs& a, cudaStream_t st) {
+  switch (sh.G) {
+    case 1: return launch_decode_fused_dg<D, 1>(sh, a, st);
+    case 2: return launch_decode_fused_dg<D, 2>(sh, a, st);
+    case 3: return launch_decode_fused_dg<D, 3>(sh, a, st);
+    case 4: return launch_decode_fused_dg<D, 4>(sh, a, st);
+    case 5: return launch_decode_fused_dg<D, 5>(sh, a, st);
+    case 6: return launch_decode_fused_dg<D, 6>(sh, a, st);
+    case 7: return launch_decode_fused_dg<D, 7>(sh, a, st);
+    case 8: return launch_decode_fused_dg<D, 8>(sh, a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+bool decode_fused_fits(const Shape& sh) {
+  return sh.G <= 8 && sh.K <= dec::kFusedMaxK && sh.NB <= dec::kFusedMaxNB;
+}
+
+cudaError_t launch_decode_fused(const Shape& sh, const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                                const int32_t* table, int n_pages, const int32_t* cl, const float* s, int32_t* idx,
+                                float* lse_s, uint16_t* o, float* lse_o, int* err, cudaStream_t st) {
+  DecodeFusedArgs a;
+  a.q = q;
+  a.kc = kc;
+  a.vc = vc;
+  a.cache_len = cl;
+  a.s = s;
+  a.table = table;
+  a.n_pages = n_pages;
+  a.idx = idx;
+  a.lse_s = lse_s;
+  a.o = o;
+  a.lse_o = lse_o;
+  a.err = err;
+  a.B = sh.B;
+  a.Hkv = sh.Hkv;
+  a.Lmax = sh.N;
+  a.K = sh.K;
+  a.gate = sh.gate;
+  a.gated = sh.gated;
+  a.outside = sh.outside;
+  a.need_lse = (lse_s != nullptr || sh.gate == SAS_GATE_LOG_SOFTMAX || sh.gate == SAS_GATE_SOFTMAX_OUTSIDE) ? 1 : 0;
+  a.scale = sh.scale;
+  return sh.d == 128 ? launch_decode_fused_d<128>(sh, a, st) : launch_decode_fused_d<64>(sh, a, st);
 }
 
 cudaError_t launch_decode_combine(const Shape& sh, int n_split, const float* o_part, const float* lse_part,

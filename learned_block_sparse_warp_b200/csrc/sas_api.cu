@@ -28,6 +28,10 @@ cudaError_t launch_decode_paged(const Shape& sh, const uint16_t* q, const uint16
                                 int* err, cudaStream_t st);
 cudaError_t launch_decode_combine(const Shape& sh, int n_split, const float* o_part, const float* lse_part,
                                   uint16_t* o, float* lse_o, cudaStream_t st);
+bool decode_fused_fits(const Shape& sh);
+cudaError_t launch_decode_fused(const Shape& sh, const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                                const int32_t* table, int n_pages, const int32_t* cl, const float* s, int32_t* idx,
+                                float* lse_s, uint16_t* o, float* lse_o, int* err, cudaStream_t st);
 cudaError_t launch_wait_timeout(int* err, cudaStream_t st);
 }  // namespace sas
 
@@ -250,6 +254,36 @@ sas_status sas_decode_combine(const sas_params* p, int n_split, const float* o_p
   if (n_split < 1 || n_split > sh.K + 1) return SAS_ERR_INVALID_ARG;
   return from_cuda(sas::launch_decode_combine(sh, n_split, o_part, lse_part, o, lse_o,
                                               static_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_decode_fused(const sas_params* p, const sas_bf16* q, const sas_bf16* kc, const sas_bf16* vc,
+                            const int32_t* cache_len, const float* s, int32_t* idx, float* lse_s, sas_bf16* o,
+                            float* lse_o, void* stream) {
+  Shape sh;
+  sas_status r = make_shape(p, &sh);
+  if (r != SAS_OK) return r;
+  if (!sas::decode_fused_fits(sh)) return SAS_ERR_UNSUPPORTED;
+  if (!ok_ptr(q) || !ok_ptr(kc) || !ok_ptr(vc) || !ok_ptr(cache_len) || !ok_ptr(s) || !ok_ptr(o) || !ok_opt(idx) ||
+      !ok_opt(lse_s) || !ok_opt(lse_o))
+    return SAS_ERR_INVALID_ARG;
+  return from_cuda(sas::launch_decode_fused(sh, q, kc, vc, nullptr, 0, cache_len, s, idx, lse_s, o, lse_o,
+                                            device_error_word(), static_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_decode_fused_paged(const sas_params* p, const sas_bf16* q, const sas_bf16* k_pages,
+                                  const sas_bf16* v_pages, int n_pages, const int32_t* block_table,
+                                  const int32_t* cache_len, const float* s, int32_t* idx, float* lse_s, sas_bf16* o,
+                                  float* lse_o, void* stream) {
+  Shape sh;
+  sas_status r = make_shape(p, &sh);
+  if (r != SAS_OK) return r;
+  if (!sas::decode_fused_fits(sh)) return SAS_ERR_UNSUPPORTED;
+  if (!ok_ptr(q) || !ok_ptr(k_pages) || !ok_ptr(v_pages) || !ok_ptr(block_table) || !ok_ptr(cache_len) ||
+      !ok_ptr(s) || !ok_ptr(o) || !ok_opt(idx) || !ok_opt(lse_s) || !ok_opt(lse_o))
+    return SAS_ERR_INVALID_ARG;
+  if (n_pages < 1 || int64_t(n_pages) * sh.Hkv > (int64_t(1) << 31) / sas::kBlock) return SAS_ERR_INVALID_ARG;
+  return from_cuda(sas::launch_decode_fused(sh, q, k_pages, v_pages, block_table, n_pages, cache_len, s, idx, lse_s,
+                                            o, lse_o, device_error_word(), static_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_selftest_wait_timeout(void* stream) {

@@ -195,6 +195,26 @@ def test_decode_split_size_limited():
     assert lib.sas_decode_paged(ctypes.byref(c), A, A, A, 8, A, A, A, A, A, 4, A, A, None) == UNSUPPORTED
 
 
+def test_decode_fused_checked():
+    # p, q, kc, vc, cache_len, s, idx, lse_s, o, lse_o, stream
+    def call(params, s=A, o=A, idx=A, cl=A):
+        return lib.sas_decode_fused(ctypes.byref(params), A, A, A, cl, s, idx, A, o, A, None)
+
+    c = _p(top_k=16, seq_len=32768).c()
+    assert call(c, s=None) == INVALID  # the scores drive the selection
+    assert call(c, o=None) == INVALID
+    assert call(c, cl=None) == INVALID
+    assert call(c, idx=A + 4) == INVALID  # misaligned optional output
+    assert call(_p(top_k=256, seq_len=32768).c()) == UNSUPPORTED  # the picks live in shared memory
+    assert call(_p(top_k=16, seq_len=64 * 4096).c()) == UNSUPPORTED  # so do the row's keys
+    assert call(_p(n_q_heads=32, n_kv_heads=2).c()) == UNSUPPORTED  # G = 16
+    paged = lib.sas_decode_fused_paged
+    # p, q, k_pages, v_pages, n_pages, table, cache_len, s, idx, lse_s, o, lse_o, stream
+    assert paged(ctypes.byref(c), A, A, A, 0, A, A, A, A, A, A, A, None) == INVALID
+    assert paged(ctypes.byref(c), A, A, A, 8, None, A, A, A, A, A, A, None) == INVALID
+    assert paged(ctypes.byref(c), A, A, A, 1 << 30, A, A, A, A, A, A, A, None) == INVALID
+
+
 def test_block_mean_keys_checked():
     c = _p().c()
     f = lib.sas_block_mean_keys
