@@ -456,7 +456,10 @@ def run_gpu(args, rank, world, local_rank):
             "combine": lambda k_: sas.sas_decode_combine(pd, n_split, o_rot[k_]["o_part"], o_rot[k_]["lse_part"],
                                                          o_rot[k_]["o"], o_rot[k_]["lse_o"], stream=stream),
             "step": lambda k_: sas.decode_step(pd, xd["q"], xd["k"], xd["v"], cl, s_rot[k_], n_split, o_rot[k_],
-                                               stream=stream)}
+                                               stream=stream),
+            # the one-launch step: select, attention and merge; a serving loop takes o and lse_o
+            "fused": lambda k_: sas.sas_decode_fused(pd, xd["q"], xd["k"], xd["v"], cl, s_rot[k_], o_rot[k_]["o"],
+                                                     lse_o=o_rot[k_]["lse_o"], stream=stream)}
 
         def capture_r(fn):
             g = torch.cuda.CUDAGraph()
@@ -465,8 +468,11 @@ def run_gpu(args, rank, world, local_rank):
                     fn(r_ % N_ROT)
             return g
 
+        with torch.cuda.stream(stream):  # the fused kernel's attributes are set outside the captures
+            kernels["fused"](0)
         graphs = {key: capture_r(fn) for key, fn in kernels.items()}
-        step_graph = sas.DecodeGraph(pd, xd["q"], xd["k"], xd["v"], cl, xd["s"], n_split, od, stream=stream)
+        step_graph = sas.DecodeGraph(pd, xd["q"], xd["k"], xd["v"], cl, xd["s"], n_split, od, stream=stream,
+                                     fused=True)
 
         def replay_timed(g):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -493,26 +499,37 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
         med = {key: statistics.median(e[0].elapsed_time(e[1]) for e in evs) / R for key, evs in timings.items()}
         med["flushed"] = statistics.median(e[0].elapsed_time(e[1]) for e in flushed)
-        step_ms = max_over_ranks(dist, med["step"], dev)
+        step_ms = max_over_ranks(dist, med["fused"], dev)
         split_ms = med["split"]
         kv = decode_kv_bytes(wd, xd["cache_len"].cpu().numpy())
-        gbs = kv / (split_ms * 1e-3) / 1e9
+        gbs = kv / (step_ms * 1e-3) / 1e9
+        split_gbs = kv / (split_ms * 1e-3) / 1e9
         line["decode"] = {
             "workload": DECODE, "tok_per_s": job_rate(wd.batch, world, step_ms * 1e-3), "ms_per_step": step_ms,
-            "launch": f"{R} steps back to back in one CUDA graph (three kernels each, chained by programmatic "
-                      f"dependent launch), rotating over {N_ROT} score sets with different selections",
+            "path": "sas_decode_fused: Top-K select, attention and LSE merge in one launch (outputs o, lse_o)",
+            "launch": f"{R} steps back to back in one CUDA graph, rotating over {N_ROT} score sets with "
+                      f"different selections",
+            "three_kernel_ms_per_step": med["step"],
+            "three_kernel": "sas_topk_select, sas_decode and sas_decode_combine chained by programmatic dependent "
+                            "launch (outputs idx, lse_s, o, lse_o)",
             "select_ms": med["select"], "split_ms": split_ms, "combine_ms": med["combine"], "n_split": n_split,
-            "breakdown": f"each kernel as {R} back-to-back launches in one graph over the rotating sets, / {R}",
+            "breakdown": f"the three-kernel path, each kernel as {R} back-to-back launches in one graph over the "
+                         f"rotating sets, / {R}",
             "flushed_ms_per_step": med["flushed"],
-            "flushed": "one captured step replayed after a 252 MB read that flushes the L2 (one graph launch "
-                       "included)",
+            "flushed": "one captured fused step replayed after a 252 MB read that flushes the L2 (one graph "
+                       "launch included)",
             "gate": "none (inference form)",
             "l2": "no flush: consecutive steps gather different blocks (rotating selections)",
-            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel (sas_decode)", "achieved": gbs,
-                         "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"], "algorithmic_bytes": kv,
-                         "traffic": traffic_record("decode_split",
+            "roofline": {"bound": "hbm", "kernel": "decode_fused_kernel (sas_decode_fused), the whole step",
+                         "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
+                         "algorithmic_bytes": kv,
+                         "traffic": traffic_record("decode_fused",
                                                    ["learned_block_sparse_warp_b200/csrc/decode.cu"])},
-            "gpu_launches_per_step": 3}
+            "split_roofline": {"kernel": "decode_split_kernel (sas_decode)", "achieved": split_gbs,
+                               "frac": split_gbs / pk["hbm"],
+                               "traffic": traffic_record("decode_split",
+                                                         ["learned_block_sparse_warp_b200/csrc/decode.cu"])},
+            "gpu_launches_per_step": 1}
         del step_graph, kernels, graphs, o_rot, s_rot
         if sas.sas_get_device_error(stream) != 0:
             raise RuntimeError("device error during decode")
@@ -574,7 +591,7 @@ def compact_summary(line: dict) -> dict:
     """Every workload's headline in a few hundred characters, three significant digits.
 
     train: [ms per step, TFLOP/s, fraction of burst bf16 peak]; fwd/bwd: [TFLOP/s, fraction];
-    decode: [tokens/s, µs per step, split-kernel GB/s, its fraction of HBM]; sweep: one
+    decode: [tokens/s, µs per step, GB/s of the one-launch step, its fraction of HBM]; sweep: one
     [top_k, seq_len, ms, TFLOP/s, fraction] per point (the 128K forward first);
     long_decode: [batch, cache tokens, µs per step, the selection's share of the kernels' time]."""
     out = {}

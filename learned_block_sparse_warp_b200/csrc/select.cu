@@ -237,7 +237,6 @@ __global__ void __launch_bounds__(kRowThreads) select_decode_cta_kernel(const fl
     const int m = tid + kRowThreads * v;
     if (m >= t) f[v] = -INFINITY;
     key[v] = (m < t) ? score_key(f[v]) + 1u : 0u;
-    asm volatile("" : "+r"(key[v]));  // held in a register, not re-read in every round of the search
     mx = fmaxf(mx, f[v]);
   }
   if (lse != nullptr) {
