@@ -17,13 +17,19 @@
 //       dVᵀ += dOᵀ P and dKᵀ += Qᵀ dZ then accumulate in TMEM as M = 128
 //       (d-major) MMAs with MN-major operands, so dK_j and dV_j stay on chip
 //       for the whole walk. The CTA is also the only writer of dl[t, slot(j)].
-//   bwd_q_sm100_kernel   one CTA per (batch, KV head, query block, head pair):
-//       the tile's Q and dO rows stay in TMEM as the A operands of S and dP,
-//       S and dP per selected block land in TMEM, dZ is written back as bf16
-//       over S, and dQ += dZ K is a TS MMA with K MN-major. dQ is written once,
-//       in bf16.
-// The first pass recomputes S and dP a second time (7 GEMM-shaped products
-// instead of 5), but no partial sum is ever sent to L2.
+//       With the full workspace it also stores every dZ tile (128 x 64 bf16
+//       per query block, attended block and head pair) by TMA.
+//   bwd_dq_sm100_kernel  (full workspace) one CTA per (batch, KV head, query
+//       block, up to two head pairs): dQ = scale · Σ_j dZ_tj K_j as a gather
+//       GEMM over the stored tiles and the attended K blocks, accumulated in
+//       TMEM and written once in bf16. It reads each tile once and computes
+//       no exponential: HBM-bound.
+//   bwd_q_sm100_kernel   (minimal workspace) the same dQ without the stored
+//       tiles: the tile's Q and dO rows stay in TMEM as the A operands of S
+//       and dP, S and dP per selected block land in TMEM, dZ is written back
+//       as bf16 over S, and dQ += dZ K is a TS MMA with K MN-major. It
+//       recomputes S and dP (7 GEMM-shaped products instead of 5) in exchange
+//       for a workspace without the tiles.
 #include "sm100.cuh"
 
 namespace sas {
