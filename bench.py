@@ -413,7 +413,7 @@ def run_gpu(args, rank, world, local_rank):
                          "traffic": traffic_record("bwd_call", ["learned_block_sparse_warp_b200/csrc/bwd_mma.cu",
                                                                 "learned_block_sparse_warp_b200/csrc/bwd_sm100.cu"])},
             "e2e": e2e,
-            "gpu_launches": args.steps * 9,
+            "gpu_launches": args.steps * 10,
             "clocks": clk.summary(),
         })
         del x, out

@@ -30,6 +30,8 @@ struct BwdWs {
   float* drow;     // [B, Hq, N]
   float* dl;       // [B, Hkv, NB, K]
   int* rev_cnt;    // [B, Hkv, NB]
+  uint32_t* col_bits;  // [B, Hkv, NB, W]: bit t of block j's row is set when idx[t] holds j (NB <= kBitmapMaxNB)
+  int* col_pre;        // [B, Hkv, NB, W]: set bits of block j's row in the words before w
   int* rev_off;    // [B, Hkv, NB + 1]
   int* rev_list;   // [B, Hkv, NB * K]: (t << kSlotBits) | slot
   float* rev_lam;  // [B, Hkv, NB * K]: log2-domain gate of each reverse-index entry
@@ -37,6 +39,12 @@ struct BwdWs {
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Up to this many blocks the reverse index is built from a bitmap of which
+// query blocks selected each block (two words of workspace per 32 blocks and
+// block); longer rows test every (t, j) pair against the row's sorted list.
+constexpr int kBitmapMaxNB = 4096;
+static int bitmap_words(const Shape& sh) { return sh.NB <= kBitmapMaxNB ? (sh.NB + 31) / 32 : 0; }
 
 long long bwd_dz_tiles(const Shape& sh);
 
@@ -59,6 +67,11 @@ size_t bwd_ws_layout(const Shape& sh, bool spill, void* base, BwdWs* ws) {
   off = align256(off + bhk * sh.NB * sh.K * sizeof(int));
   size_t o_lam = off;
   off = align256(off + bhk * sh.NB * sh.K * sizeof(float));
+  const size_t n_bits = bhk * sh.NB * size_t(bitmap_words(sh));
+  size_t o_bits = off;
+  off = align256(off + n_bits * sizeof(uint32_t));
+  size_t o_pre = off;
+  off = align256(off + n_bits * sizeof(int));
   size_t o_dz = off;
   if (spill) off = align256(off + size_t(bwd_dz_tiles(sh)) * 128 * 64 * sizeof(uint16_t));
   if (ws != nullptr) {
@@ -69,6 +82,8 @@ size_t bwd_ws_layout(const Shape& sh, bool spill, void* base, BwdWs* ws) {
     ws->rev_off = reinterpret_cast<int*>(p + o_off);
     ws->rev_list = reinterpret_cast<int*>(p + o_list);
     ws->rev_lam = reinterpret_cast<float*>(p + o_lam);
+    ws->col_bits = n_bits ? reinterpret_cast<uint32_t*>(p + o_bits) : nullptr;
+    ws->col_pre = n_bits ? reinterpret_cast<int*>(p + o_pre) : nullptr;
     ws->dz = spill ? reinterpret_cast<uint16_t*>(p + o_dz) : nullptr;
   }
   return off;
@@ -195,6 +210,73 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const int32_t* __restr
   }
 }
 
+// The same reverse index from a bitmap, with every step parallel over the
+// selection's entries or the blocks:
+//   mark     one thread per entry (b, h, t, s): j = idx[t][s] sets bit t of
+//            block j's row (a zeroed [NB, W] bitmap per (b, h));
+//   colscan  one warp per (b, h, j): the row's count of set bits, and per
+//            word the set bits before it;
+//   fill     one thread per entry: its place in j's list is j's offset plus
+//            the set bits of j's row below t, and the entry is (t, s).
+// The lists come out ascending in t, as from the pairwise kernels above.
+__global__ void __launch_bounds__(256) revidx_mark_kernel(const int32_t* __restrict__ idx, int nbh, int NB, int K,
+                                                         int W, uint32_t* __restrict__ bits) {
+  const size_t e = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= size_t(nbh) * NB * K) return;
+  const int s = int(e % K);
+  const size_t row = e / K;  // (b, h, t)
+  const int t = int(row % NB);
+  if (s >= min(K, t)) return;
+  const int j = idx[e];
+  if (j < 0 || j >= t) return;
+  const size_t bh = row / NB;
+  atomicOr(bits + (bh * NB + j) * W + (t >> 5), 1u << (t & 31));
+}
+
+__global__ void __launch_bounds__(256) revidx_colscan_kernel(const uint32_t* __restrict__ bits, int rows, int W,
+                                                            int* __restrict__ pre, int* __restrict__ cnt) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int lane = threadIdx.x & 31;
+  int run = 0;
+  for (int w0 = 0; w0 < W; w0 += 32) {
+    const int w = w0 + lane;
+    const int c = w < W ? __popc(bits[size_t(r) * W + w]) : 0;
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += u;
+    }
+    if (w < W) pre[size_t(r) * W + w] = run + incl - c;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) cnt[r] = run;
+}
+
+__global__ void __launch_bounds__(256) revidx_fill_cols_kernel(const int32_t* __restrict__ idx, int nbh, int NB, int K,
+                                                              int W, const uint32_t* __restrict__ bits,
+                                                              const int* __restrict__ pre, const int* __restrict__ off,
+                                                              int* __restrict__ list, const float* __restrict__ s,
+                                                              const float* __restrict__ lse_s, int gate,
+                                                              float* __restrict__ lam) {
+  const size_t e = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= size_t(nbh) * NB * K) return;
+  const int slot = int(e % K);
+  const size_t row = e / K;
+  const int t = int(row % NB);
+  if (slot >= min(K, t)) return;
+  const int j = idx[e];
+  if (j < 0 || j >= t) return;
+  const size_t bh = row / NB;
+  const size_t wi = (bh * NB + j) * W + (t >> 5);
+  const int pos = off[bh * (NB + 1) + j] + pre[wi] + __popc(bits[wi] & ((1u << (t & 31)) - 1u));
+  list[bh * NB * K + pos] = (t << kSlotBits) | slot;
+  if (lam != nullptr)
+    lam[bh * NB * K + pos] =
+        gate != SAS_GATE_NONE ? gate_lam2(gate, s[row * NB + j], lse_s != nullptr ? lse_s[row] : 0.f) : 0.f;
+}
+
 // One warp per (b, h, t): ds[t, m] = dl[t, m]·[m∈I] − softmax(s_t)_m Σ dl.
 __global__ void __launch_bounds__(256) bwd_ds_chain_kernel(const float* __restrict__ s, const float* __restrict__ lse_s,
                                                            const int32_t* __restrict__ idx,
@@ -263,10 +345,22 @@ static cudaError_t launch_bwd_d(const Shape& sh, const uint16_t* q, const uint16
     bwd_prep_kernel<D><<<std::max(1u, grid), 256, 0, st>>>(o, dO, rows_q, ws.drow);
   }
   const int nw = nbh * sh.NB;
-  revidx_count_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_cnt);
-  revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
-  revidx_fill_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_off, ws.rev_list, s, lse_s,
-                                                    sh.gate, ws.rev_lam);
+  const int W = bitmap_words(sh);
+  if (W > 0) {
+    const size_t n_ent = size_t(nw) * sh.K;
+    const unsigned ent_blocks = unsigned((n_ent + 255) / 256);
+    if ((e = cudaMemsetAsync(ws.col_bits, 0, size_t(nw) * W * sizeof(uint32_t), st)) != cudaSuccess) return e;
+    revidx_mark_kernel<<<ent_blocks, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, W, ws.col_bits);
+    revidx_colscan_kernel<<<(nw + 7) / 8, 256, 0, st>>>(ws.col_bits, nw, W, ws.col_pre, ws.rev_cnt);
+    revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
+    revidx_fill_cols_kernel<<<ent_blocks, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, W, ws.col_bits, ws.col_pre,
+                                                        ws.rev_off, ws.rev_list, s, lse_s, sh.gate, ws.rev_lam);
+  } else {
+    revidx_count_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_cnt);
+    revidx_scan_kernel<<<nbh, 32, 0, st>>>(ws.rev_cnt, sh.NB, ws.rev_off);
+    revidx_fill_kernel<<<(nw + 7) / 8, 256, 0, st>>>(idx, nbh, sh.NB, sh.K, ws.rev_off, ws.rev_list, s, lse_s,
+                                                      sh.gate, ws.rev_lam);
+  }
   // tcgen05 passes: dK/dV/dl (and the dZ tiles) KV-major, then dQ query-major
   if ((e = launch_bwd_passes_sm100(sh, q, k, v, dO, s, idx, lse_s, lse_o, ws.drow, ws.rev_off, ws.rev_list,
                                    ws.rev_lam, ws.dl, ws.dz, dq, dk, dv, err, st)) != cudaSuccess)

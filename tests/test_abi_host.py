@@ -101,9 +101,12 @@ def test_workspace_size_and_check():
     n_min = sas.sas_bwd_workspace_size_min(p)
     n = sas.sas_bwd_workspace_size(p)
     B, Hq, Hkv, N, d, NB, K = 2, 8, 2, 2048, 128, 32, 8
-    # D rows, dl, the reverse index (counts, offsets, entries, gates); no fp32 dQ at d = 128
-    lower = 4 * (B * Hq * N + B * Hkv * NB * K) + 4 * (B * Hkv * NB * 2 + 2 * B * Hkv * NB * K)
-    assert lower <= n_min <= lower + 7 * 256
+    # D rows, dl, the reverse index (counts, offsets, entries, gates) and the selection bitmap with
+    # its per-word prefix counts (one word each per 32 blocks and row); no fp32 dQ at d = 128
+    W = (NB + 31) // 32
+    lower = 4 * (B * Hq * N + B * Hkv * NB * K) + 4 * (B * Hkv * NB * 2 + 2 * B * Hkv * NB * K) \
+        + 8 * B * Hkv * NB * W
+    assert lower <= n_min <= lower + 9 * 256
     # the full size adds one 16 KB dZ tile per (batch, KV head, query block, attended block, head pair)
     tiles = B * Hkv * sum(1 + min(K, t) for t in range(NB)) * ((Hq // Hkv + 1) // 2)
     assert n_min + tiles * 16384 <= n <= n_min + tiles * 16384 + 256
