@@ -676,6 +676,8 @@ def sweep_section(args, sas, stream, dev, pk, dist, world):
             x = sweep_inputs(w, dev, torch)
         torch.cuda.synchronize()
         out = sas.empty_prefill_outputs(p, device=dev, backward=w.backward)
+        if w.backward and args.min_workspace:  # the smallest workspace: dQ recomputes S and dP
+            out["ws"] = torch.empty((sas.sas_bwd_workspace_size_min(p),), dtype=torch.uint8, device=dev)
 
         def run(evs=None):
             # select + LSE, forward, backward; with evs, an event after each call
@@ -722,7 +724,8 @@ def sweep_section(args, sas, stream, dev, pk, dist, world):
                        "ms_per_step": ms, "tflops": tf, "frac": tf / (pk["bf16"] * world),
                        "breakdown_ms": split_ms,
                        "fwd_tflops": F / (split_ms["fwd"] * 1e-3) / 1e12,
-                       "bwd_tflops": 2.5 * F / (split_ms["bwd"] * 1e-3) / 1e12 if w.backward else None})
+                       "bwd_tflops": 2.5 * F / (split_ms["bwd"] * 1e-3) / 1e12 if w.backward else None,
+                       "bwd_workspace": ("minimal" if args.min_workspace else "full") if w.backward else None})
         del x, out
         torch.cuda.empty_cache()
     return {"points": points, "peak": pk["bf16"], "peak_source": pk["source"] + " burst bf16",
@@ -882,6 +885,8 @@ def main():
                     help="run only one workload (for profiling); the JSON line needs 'all'")
     ap.add_argument("--n-split", type=int, default=0, help="decode splits (0: K + 1)")
     ap.add_argument("--sweep-point", default="", help="with --only sweep: run this sweep workload alone (profiling)")
+    ap.add_argument("--min-workspace", action="store_true",
+                    help="with --only sweep: give sas_bwd its smallest workspace (the recomputing dQ pass)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
