@@ -185,3 +185,26 @@ def test_decode_fused_limits_and_bad_length():
     torch.cuda.synchronize()
     assert sas.sas_get_device_error() == 6  # SAS_ERR_DEVICE_INDEX
     assert np.isfinite(host(o)).all()
+
+
+def test_decode_fused_paged_bad_page_is_reported():
+    """A table entry outside the page pool for a block the step reads raises the device error
+    word; the kernel reads page 0 in its place and the output stays finite."""
+    sas = _sas()
+    B, Hq, Hkv, d, Lmax, K = 2, 8, 2, 128, 1024, 4
+    q, kc, vc, s = _case(B, Hq, Hkv, d, Lmax, seed=15)
+    g = np.random.default_rng(19)
+    lens = [700, 1024]
+    kp, vp, table = _paged(kc, vc, lens, g, n_extra=0)
+    kp = np.nan_to_num(kp)  # every page is read-safe here; only the table entry is wrong
+    vp = np.nan_to_num(vp)
+    table[1, (lens[1] - 1) // 64] = kp.shape[0] + 3  # the current block of sequence 1
+    p = sas.Params(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=Lmax, top_k=K,
+                   gate_mode=O.GATE_NONE)
+    o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device="cuda")
+    sas.sas_decode_fused_paged(p, bf16_dev(q), bf16_dev(kp), bf16_dev(vp), torch.from_numpy(table).cuda(),
+                               torch.tensor(lens, dtype=torch.int32).cuda(), f32_dev(s), o)
+    torch.cuda.synchronize()
+    assert sas.sas_get_device_error() == 6  # SAS_ERR_DEVICE_INDEX
+    assert sas.sas_get_device_error() == 0  # read and cleared
+    assert np.isfinite(host(o)).all()
