@@ -505,6 +505,11 @@ __global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFused
     asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(sP + i * 16), "r"(0));
   griddep_wait();  // q, the caches, the scores and cache_len may come from the work just before
 
+  // the row's scores are read while the cache length is still in flight
+  const float* srow = a.s + size_t(bh) * NB;
+  uint32_t* key_s = reinterpret_cast<uint32_t*>(smem + (STAGES - 1) * STAGEB);
+  int* hist_s = reinterpret_cast<int*>(key_s + dec::kFusedMaxNB);
+  for (int m = tid; m < NB - 1; m += dec::kThreads) key_s[m] = __float_as_uint(__ldg(srow + m));
   int L = a.cache_len[b];
   if (L < 1 || L > a.Lmax) {
     if (tid == 0) raise_error(a.err, SAS_ERR_DEVICE_INDEX);
@@ -512,7 +517,6 @@ __global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFused
   }
   const int c = (L - 1) / kBlock;  // the current block; history blocks are [0, c)
   const int n = min(a.K, c);
-  const float* srow = a.s + size_t(bh) * NB;
 
   // ---- this CTA's share of the ordered list [c, picks...]
   const int nl = 1 + n;
@@ -557,11 +561,9 @@ __global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFused
     cp_async_commit();
   }
   // ---- selection: keys of the history scores in the last ring stage (not loaded before the loop)
-  uint32_t* key_s = reinterpret_cast<uint32_t*>(smem + (STAGES - 1) * STAGEB);
-  int* hist_s = reinterpret_cast<int*>(key_s + dec::kFusedMaxNB);
   float mx = -INFINITY;
-  for (int m = tid; m < c; m += dec::kThreads) {
-    const float v = __ldg(srow + m);
+  for (int m = tid; m < c; m += dec::kThreads) {  // each thread converts the scores it read
+    const float v = __uint_as_float(key_s[m]);
     key_s[m] = score_key(v) + 1u;  // >= 1, so the threshold 1 takes every block
     mx = fmaxf(mx, v);
   }
@@ -585,9 +587,12 @@ __global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFused
   const bool all = (n == c), none = (n == 0);
   int need_eq = 0, eq_cnt = 0;
   const uint32_t thr = (all || none) ? 1u : cta_kth_key(key_s, c, n, hist_s, xch_s, need_eq, eq_cnt);
-  if (!none && (all || need_eq == eq_cnt)) {
+  int32_t* idx_row = (rank == 0 && a.idx != nullptr) ? a.idx + size_t(bh) * a.K : nullptr;
+  const bool fast = !none && (all || need_eq == eq_cnt);
+  if (fast) {
     // no tie is cut at the threshold: the picks are exactly the keys >= thr. They
-    // are appended in any order, then each is placed by the number of smaller picks.
+    // are appended in any order, then each is placed by the number of smaller
+    // picks, and its thread also writes it out and looks up its gate.
     int* app_s = hist_s + 256;
     for (int m = tid; m < c; m += dec::kThreads)
       if (key_s[m] >= thr) app_s[atomicAdd(&napp_s, 1)] = m;
@@ -597,6 +602,9 @@ __global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFused
       int r = 0;
       for (int j = 0; j < n; ++j) r += app_s[j] < v ? 1 : 0;
       sel_s[r] = v;
+      if (idx_row != nullptr) idx_row[r] = v;
+      const int jt = r + 1 - p0;  // this CTA's task at list position r + 1
+      if (jt >= 0 && jt < nt) lam_s[jt] = a.gated ? gate_lam2(a.gate, __ldg(srow + v), lse) : 0.f;
     }
   } else if (!none) {
     // ties cut at the threshold, taken from the lowest block index: each thread
@@ -622,17 +630,17 @@ __global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFused
       e += is_eq ? 1 : 0;
     }
   }
-  __syncthreads();
-  if (rank == 0) {
-    if (a.idx != nullptr)
-      for (int i = tid; i < a.K; i += dec::kThreads) a.idx[size_t(bh) * a.K + i] = i < n ? sel_s[i] : -1;
-    if (a.lse_s != nullptr && tid == 0) a.lse_s[bh] = lse;
+  if (idx_row != nullptr)
+    for (int i = n + tid; i < a.K; i += dec::kThreads) idx_row[i] = -1;
+  if (rank == 0 && a.lse_s != nullptr && tid == 0) a.lse_s[bh] = lse;
+  if (p0 == 0 && nt > 0 && tid == 0) lam_s[0] = 0.f;  // the current block takes no gate
+  __syncthreads();  // the picks are placed, and the keys' stage is free for the ring
+  if (!fast && !none) {  // the tie path placed the picks by block scans: write them out and take their gates
+    if (idx_row != nullptr)
+      for (int i = tid; i < n; i += dec::kThreads) idx_row[i] = sel_s[i];
+    for (int j = tid; j < nt; j += dec::kThreads)
+      if (p0 + j > 0) lam_s[j] = a.gated ? gate_lam2(a.gate, __ldg(srow + sel_s[p0 + j - 1]), lse) : 0.f;
   }
-  for (int j = tid; j < nt; j += dec::kThreads) {
-    const int pos = p0 + j;
-    lam_s[j] = (pos > 0 && a.gated) ? gate_lam2(a.gate, __ldg(srow + sel_s[pos - 1]), lse) : 0.f;
-  }
-  __syncthreads();  // lam_s is written, and the keys' stage is free for the ring
 
   DecAcc<D> acc;
 #pragma unroll
