@@ -408,61 +408,107 @@ __device__ __forceinline__ int cta_excl_sum(int v, int* wtot, int& tot) {
   return before;
 }
 
-// The n-th largest of key[0, c) in shared memory (0 < n < c), by four 8-bit
-// radix passes from the most significant byte: each pass histograms the keys
-// that match the digits fixed so far and fixes the digit at which the count
-// from the top reaches the number still needed. Returns the threshold key;
-// need_eq gets how many keys equal to it belong to the n largest, and eq_cnt
-// how many keys equal it. (Plain shared atomics: aggregating equal digits
-// within a warp first, by match.any, measured slower on sm_100a.)
-__device__ uint32_t cta_kth_key(const uint32_t* key, int c, int n, int* hist, int* xch, int& need_eq, int& eq_cnt) {
+// One 8-bit radix pass over the keys of key[0, c) whose bits above `shift + 8`
+// equal prefix's: fixes the digit at which the count from the top bin reaches
+// need. xch gets the digit, the number still needed within its bin, and the
+// bin's count. (Plain shared atomics: aggregating equal digits within a warp
+// first, by match.any, measured slower on sm_100a.)
+__device__ void cta_radix_pass(const uint32_t* key, int c, int pass, uint32_t prefix, int need, int* hist, int* xch) {
   const int tid = threadIdx.x, lane = tid & 31;
-  uint32_t prefix = 0u;
-  int need = n;
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += dec::kThreads) hist[i] = 0;
-    __syncthreads();
-    for (int m = tid; m < c; m += dec::kThreads) {
-      const uint32_t k = key[m];
-      if (pass == 0 || ((k ^ prefix) >> (shift + 8)) == 0u) atomicAdd(&hist[(k >> shift) & 255u], 1);
+  const int shift = 24 - 8 * pass;
+  for (int i = tid; i < 256; i += dec::kThreads) hist[i] = 0;
+  __syncthreads();
+  for (int m = tid; m < c; m += dec::kThreads) {
+    const uint32_t k = key[m];
+    if (pass == 0 || ((k ^ prefix) >> (shift + 8)) == 0u) atomicAdd(&hist[(k >> shift) & 255u], 1);
+  }
+  __syncthreads();
+  if (tid < 32) {  // lane owns bins [8 lane, 8 lane + 8); counts run from the top bin down
+    int cnt[8], own = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      cnt[u] = hist[8 * lane + u];
+      own += cnt[u];
     }
-    __syncthreads();
-    if (tid < 32) {  // lane owns bins [8 lane, 8 lane + 8); counts run from the top bin down
-      int cnt[8], own = 0;
+    int incl = own;  // own plus every lane above
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        cnt[u] = hist[8 * lane + u];
-        own += cnt[u];
-      }
-      int incl = own;  // own plus every lane above
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_down_sync(0xffffffffu, incl, off);
+      if (lane + off < 32) incl += u;
+    }
+    int acc = incl - own;  // keys in bins above this lane's
+    if (acc < need && need <= incl) {
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int u = __shfl_down_sync(0xffffffffu, incl, off);
-        if (lane + off < 32) incl += u;
-      }
-      int acc = incl - own;  // keys in bins above this lane's
-      if (acc < need && need <= incl) {
-#pragma unroll
-        for (int u = 7; u >= 0; --u) {
-          if (acc + cnt[u] >= need) {
-            xch[0] = 8 * lane + u;
-            xch[1] = need - acc;
-            xch[2] = cnt[u];
-            break;
-          }
-          acc += cnt[u];
+      for (int u = 7; u >= 0; --u) {
+        if (acc + cnt[u] >= need) {
+          xch[0] = 8 * lane + u;
+          xch[1] = need - acc;
+          xch[2] = cnt[u];
+          break;
         }
+        acc += cnt[u];
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// The n largest of key[0, c) in shared memory (0 < n < c), ties to the lowest
+// index. The first 8-bit radix pass fixes the leading byte of the n-th largest
+// key. When at most 128 keys share that byte (the usual case: scores spread
+// over several exponents), those candidates are ranked against each other
+// directly, one per thread, and the picks (every key with a larger leading
+// byte, and the candidates ranked below the number still needed) are appended
+// to app in any order. Otherwise three more passes find the exact threshold;
+// the picks are appended likewise unless a tie is cut at it, in which case
+// the function returns true with the threshold and the number of its equals
+// to take, and the caller places the picks in index order.
+__device__ bool cta_select(const uint32_t* key, int c, int n, int* hist, int* xch, int* app, int* napp,
+                           uint32_t* cand_k, int* cand_m, int* ncand, uint32_t& thr, int& need_eq) {
+  const int tid = threadIdx.x;
+  if (tid == 0) *ncand = 0;
+  cta_radix_pass(key, c, 0, 0u, n, hist, xch);
+  const uint32_t d0 = uint32_t(xch[0]);
+  const int need1 = xch[1], cnt0 = xch[2];
+  if (cnt0 <= dec::kThreads) {
+    for (int m = tid; m < c; m += dec::kThreads) {
+      const uint32_t k = key[m], top = k >> 24;
+      if (top > d0) {
+        app[atomicAdd(napp, 1)] = m;
+      } else if (top == d0) {
+        const int s = atomicAdd(ncand, 1);
+        cand_k[s] = k;
+        cand_m[s] = m;
       }
     }
     __syncthreads();
-    prefix |= uint32_t(xch[0]) << shift;
+    if (tid < cnt0) {
+      const uint32_t k = cand_k[tid];
+      const int mi = cand_m[tid];
+      int r = 0;  // candidates ahead of this one: larger keys, and equal keys at lower indexes
+#pragma unroll 8
+      for (int j = 0; j < cnt0; ++j) {
+        const uint32_t kj = cand_k[j];
+        r += (kj > k || (kj == k && cand_m[j] < mi)) ? 1 : 0;
+      }
+      if (r < need1) app[atomicAdd(napp, 1)] = mi;
+    }
+    return false;
+  }
+  uint32_t prefix = d0 << 24;
+  int need = need1;
+#pragma unroll 1
+  for (int pass = 1; pass < 4; ++pass) {
+    cta_radix_pass(key, c, pass, prefix, need, hist, xch);
+    prefix |= uint32_t(xch[0]) << (24 - 8 * pass);
     need = xch[1];
   }
+  thr = prefix;
   need_eq = need;
-  eq_cnt = xch[2];
-  return prefix;
+  if (need_eq != xch[2]) return true;  // a tie is cut at the threshold
+  for (int m = tid; m < c; m += dec::kThreads)
+    if (key[m] >= thr) app[atomicAdd(napp, 1)] = m;
+  return false;
 }
 
 template <int D, int G, int STAGES>
@@ -473,11 +519,11 @@ __global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFused
   constexpr int QB = 16 * ROWB;
   constexpr int STAGEB = 2 * TILEB + QB;
   constexpr int DW = D / 4;
-  static_assert(dec::kFusedMaxNB * 4 + 512 * 4 <= STAGEB, "keys, histogram and picks fit one ring stage");
+  static_assert(dec::kFusedMaxNB * 4 + 768 * 4 <= STAGEB, "keys, histogram, picks and candidates fit one ring stage");
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int sel_s[dec::kFusedMaxK];         // the row's picks, ascending
   __shared__ float lam_s[dec::kFusedMaxK + 1];   // log2 gate of each of this CTA's tasks
-  __shared__ int xch_s[3], wtot_s[dec::kThreads / 32], napp_s;
+  __shared__ int xch_s[4], wtot_s[dec::kThreads / 32], napp_s;
   __shared__ float redf_s[dec::kThreads / 32];
   __shared__ float red_max[4][8], red_sum[4][8];
   __shared__ __align__(128) uint16_t p_s[16 * kBlock];
@@ -585,17 +631,20 @@ __global__ void __launch_bounds__(dec::kThreads) decode_fused_kernel(DecodeFused
   }
   __syncthreads();  // every key is in place
   const bool all = (n == c), none = (n == 0);
-  int need_eq = 0, eq_cnt = 0;
-  const uint32_t thr = (all || none) ? 1u : cta_kth_key(key_s, c, n, hist_s, xch_s, need_eq, eq_cnt);
+  int need_eq = 0;
+  uint32_t thr = 1u;
   int32_t* idx_row = (rank == 0 && a.idx != nullptr) ? a.idx + size_t(bh) * a.K : nullptr;
-  const bool fast = !none && (all || need_eq == eq_cnt);
+  int* app_s = hist_s + 256;
+  uint32_t* cand_k = reinterpret_cast<uint32_t*>(app_s + 256);
+  int* cand_m = app_s + 384;
+  bool tie = false;
+  if (all) {
+    for (int m = tid; m < c; m += dec::kThreads) app_s[m] = m;
+  } else if (!none) {
+    tie = cta_select(key_s, c, n, hist_s, xch_s, app_s, &napp_s, cand_k, cand_m, &xch_s[3], thr, need_eq);
+  }
+  const bool fast = !none && !tie;
   if (fast) {
-    // no tie is cut at the threshold: the picks are exactly the keys >= thr. They
-    // are appended in any order, then each is placed by the number of smaller
-    // picks, and its thread also writes it out and looks up its gate.
-    int* app_s = hist_s + 256;
-    for (int m = tid; m < c; m += dec::kThreads)
-      if (key_s[m] >= thr) app_s[atomicAdd(&napp_s, 1)] = m;
     __syncthreads();
     for (int i = tid; i < n; i += dec::kThreads) {
       const int v = app_s[i];
